@@ -1,0 +1,381 @@
+#!/usr/bin/env python
+"""Tree-verify step benchmark (one B200 per process).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kd|reference]
+
+A step is one pass of the whole verify path over one batch: node-latent write,
+mask build, MLA-absorb tree attention (tensor cores), greedy accept and
+compaction, for the 64-request loop workload (64 heads, 17 tree nodes, cache
+lengths U[2048, 16384]).  Each rank verifies its own 64 requests (weak scaling;
+no collective on the data path).  Prints one JSON line on rank 0.
+
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the
+same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from tree_speculative_decoding_kd_b200 import harness as HN  # noqa: E402
+from tree_speculative_decoding_kd_b200 import workload as W  # noqa: E402
+
+METRIC = "tree-verify MLA attn TFLOP/s + KV HBM GB/s (% roofline); verify steps/s"
+N_DISTINCT = 8          # distinct pre-generated step inputs, cycled
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["kd", "reference"], default="kd")
+    ap.add_argument("--no-extras", action="store_true", help="skip the per-config attention lines")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_cfg(rank: int, steps_total: int):
+    cfg = W.CONFIGS["loop"]
+    return W.scaled(cfg, seed=HN.rank_seed(cfg.seed, rank), steps=max(cfg.steps, steps_total))
+
+
+def config_json(cfg):
+    return {"workload": f"loop: {cfg.B} requests x {cfg.H} heads, d_c=512 d_r=64 bf16, "
+                        f"{cfg.n} tree nodes (depth<=8), L~U[{cfg.L_lo},{cfg.L_hi}], "
+                        "write-nodes+mask+verify+accept+compact per step",
+            "requests_per_gpu": cfg.B, "heads": cfg.H, "tree_nodes": cfg.n,
+            "cache_len": [cfg.L_lo, cfg.L_hi], "scale": cfg.scale,
+            "l2": "inputs larger than L2 (each step reads ~0.8 GB of latent cache)",
+            "step_inputs": f"{N_DISTINCT} distinct seeded step inputs cycled"}
+
+
+# ====================================================================== CPU oracle
+def oracle_step_sample(wl_c, wl_r, lens, st, cfg, reqs):
+    """Oracle time of one step, measured on `reqs` requests' attention and
+    compaction plus every request's accept, extrapolated to all requests."""
+    import oracle
+    from oracle.accept import tree_accept_batch
+    t0 = time.perf_counter()
+    vis = np.stack([oracle.visibility_words(p) for p in st.parents])
+    path, ln, _ = tree_accept_batch(st.tokens, st.parents, st.argmax)
+    t_all = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    for b in reqs:
+        sl = slice(b, b + 1)
+        c1, r1 = oracle.kv_write_nodes(wl_c[sl], wl_r[sl], lens[sl], st.node_ckv[sl], st.node_krope[sl])
+        oracle.tree_verify_attention(st.q_abs[sl], st.q_rope[sl], c1, r1, lens[sl], vis[sl], cfg.scale)
+        oracle.kv_compact(c1, r1, lens[sl], path[sl], ln[sl])
+    t_req = (time.perf_counter() - t1) / len(reqs)
+    return t_all + t_req * cfg.B
+
+
+def cpu_baseline(cfg, wl, st, budget_s=12.0):
+    """The oracle as it stands, timed on this host's cores on a bounded sample."""
+    threads, api = HN.blas_threads()
+    reqs, times = [], []
+    t_start = time.perf_counter()
+    b = 0
+    while b < cfg.B and (time.perf_counter() - t_start) < budget_s:
+        times.append(oracle_step_sample(wl.c_kv, wl.k_rope, wl.cache_lens, st, cfg, [b]))
+        reqs.append(b)
+        b += 1
+    sec = float(np.median(times))
+    return {"value": 1.0 / sec, "unit": "verify steps/s", "cores": threads, "kind": "oracle",
+            "sample": f"float64 numpy oracle ({api} BLAS): attention+node write+compaction of "
+                      f"{len(reqs)} of {cfg.B} requests of step 0 (one at a time) plus accept of "
+                      f"all {cfg.B}, extrapolated to the full 64-request step"}
+
+
+def run_reference(args):
+    rank, world, _ = HN.dist_env()
+    if rank != 0:
+        return
+    cfg = workload_cfg(0, args.steps + args.warmup)
+    threads, api = HN.blas_threads()
+    wl = W.make_loop_state(cfg)
+    lens = wl.cache_lens.copy()
+    times = []
+    for s in range(args.warmup + args.steps):
+        st = W.draw_step(cfg, s % N_DISTINCT, with_nodes=True)
+        b = s % cfg.B
+        t = oracle_step_sample(wl.c_kv, wl.k_rope, lens, st, cfg, [b])
+        if s >= args.warmup:
+            times.append(t)
+    sec = float(np.sum(times))
+    value = args.steps / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "verify steps/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_json(cfg),
+            "cpu_baseline": {"value": value, "unit": "verify steps/s", "cores": threads,
+                             "kind": "oracle",
+                             "sample": f"per step: one request's attention, node write and "
+                                       f"compaction (rotating) plus all {cfg.B} accepts, "
+                                       f"extrapolated to {cfg.B} requests ({api} BLAS)"},
+            "e2e": {"value": value, "unit": "verify steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ====================================================================== GPU path
+class DeviceStep:
+    """One step's inputs on the device."""
+
+    def __init__(self, kd, st, torch):
+        self.q_abs = kd.bf16_from_bits(st.q_abs)
+        self.q_rope = kd.bf16_from_bits(st.q_rope)
+        self.node_ckv = kd.bf16_from_bits(st.node_ckv)
+        self.node_krope = kd.bf16_from_bits(st.node_krope)
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).cuda()  # noqa: E731
+        self.parents, self.tokens, self.argmax = i32(st.parents), i32(st.tokens), i32(st.argmax)
+        self.depth = np.stack([np.asarray(_depths(p)) for p in st.parents])
+
+    def tensors(self):
+        return [self.q_abs, self.q_rope, self.node_ckv, self.node_krope, self.parents,
+                self.tokens, self.argmax]
+
+
+def _depths(parents):
+    d = [0] * len(parents)
+    for i in range(1, len(parents)):
+        d[i] = d[parents[i]] + 1
+    return d
+
+
+class Verifier:
+    """The five library calls of one verify step on persistent device buffers."""
+
+    def __init__(self, kd, torch, cfg, c_kv, k_rope, lens):
+        self.kd, self.torch, self.cfg = kd, torch, cfg
+        B, n, H = cfg.B, cfg.n, cfg.H
+        self.c_kv, self.k_rope, self.lens = c_kv, k_rope, lens
+        dev = c_kv.device
+        self.err = kd.new_error_word(dev)
+        self.ws = kd.new_workspace(B, n, H, cfg.cap, 0, dev)
+        self.vis = torch.empty(B, n, (n + 31) // 32, dtype=torch.int32, device=dev)
+        self.depth = torch.empty(B, n, dtype=torch.int32, device=dev)
+        self.out = torch.empty(B, n, H, 512, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(B, n, H, dtype=torch.float32, device=dev)
+        self.path = torch.empty(B, n, dtype=torch.int32, device=dev)
+        self.len = torch.empty(B, dtype=torch.int32, device=dev)
+        self.bonus = torch.empty(B, dtype=torch.int32, device=dev)
+        self.launches_per_step = 5 + (1 if self._splits() > 1 else 0)
+
+    def _splits(self):
+        return 1 if self.kd.kd_verify_workspace_bytes(self.cfg.B, self.cfg.n, self.cfg.H,
+                                                      self.cfg.cap, 0) <= 256 else 2
+
+    def step(self, s: DeviceStep, ev=None):
+        kd = self.kd
+        kd.kd_kv_write_nodes(self.c_kv, self.k_rope, self.lens, s.node_ckv, s.node_krope, self.err)
+        kd.kd_tree_build_mask(s.parents, self.vis, self.depth, self.err)
+        if ev is not None:
+            ev[0].record()
+        kd.kd_tree_verify_attn(s.q_abs, s.q_rope, self.c_kv, self.k_rope, self.lens, self.vis,
+                               None, self.cfg.scale, self.out, self.lse, self.ws)
+        if ev is not None:
+            ev[1].record()
+        kd.kd_tree_accept(s.tokens, s.parents, s.argmax, self.path, self.len, self.bonus, self.err)
+        kd.kd_kv_compact(self.c_kv, self.k_rope, self.path, self.len, self.lens, self.err)
+
+
+def attn_extras(kd, torch, peaks, flush):
+    """Attention-only timings of the single-step configurations (parity cases)."""
+    res = {}
+    for name in ["tiny", "kimi_single", "batched", "long"]:
+        wl = W.make_workload(name)
+        cfg, st = wl.cfg, wl.step
+        qa, qr = kd.bf16_from_bits(st.q_abs), kd.bf16_from_bits(st.q_rope)
+        ck, kr = kd.bf16_from_bits(wl.c_kv), kd.bf16_from_bits(wl.k_rope)
+        lens = torch.from_numpy(wl.cache_lens.astype(np.int32)).cuda()
+        parents = torch.from_numpy(st.parents).cuda()
+        vis, _ = kd.kd_tree_build_mask(parents)
+        ws = kd.new_workspace(cfg.B, cfg.n, cfg.H, cfg.cap)
+        out = torch.empty(cfg.B, cfg.n, cfg.H, 512, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(cfg.B, cfg.n, cfg.H, dtype=torch.float32, device="cuda")
+        call = lambda: kd.kd_tree_verify_attn(qa, qr, ck, kr, lens, vis, None, cfg.scale, out, lse, ws)  # noqa: E731
+        for _ in range(3):
+            call()
+        times = []
+        for _ in range(20):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e-3)
+        t = float(np.median(times))
+        depths = [_depths(p) for p in st.parents]
+        fl = HN.attn_flops(wl.cache_lens, depths, cfg.H)
+        by = HN.attn_bytes(wl.cache_lens, cfg.n, cfg.H)
+        roof_t = max(fl / (peaks["bf16_tflops"] * 1e12), by / (peaks["hbm_gbs"] * 1e9))
+        res[name] = {"us": round(t * 1e6, 2), "tflops": round(fl / t / 1e12, 1),
+                     "hbm_gbs": round(by / t / 1e9, 1), "roofline_frac": round(roof_t / t, 3),
+                     "bound": "tensor" if fl / (peaks["bf16_tflops"] * 1e12) > by / (peaks["hbm_gbs"] * 1e9) else "hbm",
+                     "l2": "flushed (256 MB write) before each rep"}
+        del qa, qr, ck, kr, ws, out
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_kd(args):
+    import torch
+
+    rank, world, local = HN.dist_env()
+    torch.cuda.set_device(local)
+    HN.init_dist("nccl" if world > 1 else "gloo")
+    from tree_speculative_decoding_kd_b200 import kd
+
+    peaks = HN.load_peaks(ROOT)
+    cfg = workload_cfg(rank, args.steps + args.warmup)
+    wl = W.make_loop_state(cfg)
+    host_steps = [W.draw_step(cfg, s, with_nodes=True) for s in range(N_DISTINCT)]
+    dsteps = [DeviceStep(kd, st, torch) for st in host_steps]
+    c0 = kd.bf16_from_bits(wl.c_kv)
+    r0 = kd.bf16_from_bits(wl.k_rope)
+    lens0 = torch.from_numpy(wl.cache_lens.astype(np.int32)).cuda()
+
+    # ---------------- device-resident arm
+    c_kv, k_rope, lens = c0.clone(), r0.clone(), lens0.clone()
+    V = Verifier(kd, torch, cfg, c_kv, k_rope, lens)
+    for s in range(args.warmup):
+        V.step(dsteps[s % N_DISTINCT])
+    torch.cuda.synchronize()
+    # cache lengths each timed step starts from: the generator knows every
+    # step's accepted length (its planted path), so no device copy is timed
+    lens_np = wl.cache_lens.astype(np.int64).copy()
+    step_lens = []
+    for s in range(args.warmup + args.steps):
+        if s >= args.warmup:
+            step_lens.append(lens_np.copy())
+        lens_np += np.array([len(p) for p in host_steps[s % N_DISTINCT].planted])
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    HN.barrier(local)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with HN.ClockSampler(local) as clk:
+        t0.record()
+        for s in range(args.steps):
+            V.step(dsteps[(args.warmup + s) % N_DISTINCT], attn_ev[s])
+        t1.record()
+        torch.cuda.synchronize()
+    HN.barrier(local)
+    elapsed = t0.elapsed_time(t1) * 1e-3
+    elapsed_max = HN.max_over_ranks(elapsed, torch.device("cuda", local))
+    attn_times = [a.elapsed_time(b) * 1e-3 for a, b in attn_ev]
+    flop_steps, byte_steps = [], []
+    for s in range(args.steps):
+        depths = dsteps[(args.warmup + s) % N_DISTINCT].depth
+        flop_steps.append(HN.attn_flops(step_lens[s], depths, cfg.H))
+        byte_steps.append(HN.attn_bytes(step_lens[s], cfg.n, cfg.H))
+    assert np.array_equal(V.lens.cpu().numpy(), lens_np), "cache lengths diverged from the planted paths"
+    err_bits = kd.kd_read_device_error(V.err) | kd.kd_read_device_error(V.ws)
+    attn_avg = float(np.mean(attn_times))
+    flop_avg, byte_avg = float(np.mean(flop_steps)), float(np.mean(byte_steps))
+    steps_per_s = HN.whole_job_rate(args.steps, world, elapsed_max)
+
+    # ---------------- end-to-end arm: host inputs copied in, results copied out, every step
+    c_kv.copy_(c0)
+    k_rope.copy_(r0)
+    lens.copy_(lens0)
+    pinned = []
+    for ds in dsteps:
+        pinned.append([t.cpu().pin_memory() for t in ds.tensors()])
+    stage = DeviceStep.__new__(DeviceStep)
+    stage.q_abs, stage.q_rope, stage.node_ckv, stage.node_krope, stage.parents, stage.tokens, \
+        stage.argmax = [t.clone() for t in dsteps[0].tensors()]
+    res_host = [torch.empty(cfg.B, cfg.n, dtype=torch.int32).pin_memory(),
+                torch.empty(cfg.B, dtype=torch.int32).pin_memory(),
+                torch.empty(cfg.B, dtype=torch.int32).pin_memory()]
+    h2d = sum(t.numel() * t.element_size() for t in pinned[0])
+    d2h = sum(t.numel() * t.element_size() for t in res_host)
+
+    def e2e_step(s):
+        for dst, src in zip(stage.tensors(), pinned[s % N_DISTINCT]):
+            dst.copy_(src, non_blocking=True)
+        V.step(stage)
+        for dst, src in zip(res_host, (V.path, V.len, V.bonus)):
+            dst.copy_(src, non_blocking=True)
+
+    for s in range(args.warmup):
+        e2e_step(s)
+    torch.cuda.synchronize()
+    HN.barrier(local)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(args.steps):
+        e2e_step(args.warmup + s)
+    e1.record()
+    torch.cuda.synchronize()
+    HN.barrier(local)
+    e2e_el = HN.max_over_ranks(e0.elapsed_time(e1) * 1e-3, torch.device("cuda", local))
+    e2e_rate = HN.whole_job_rate(args.steps, world, e2e_el)
+
+    extras = None
+    cpu = None
+    if rank == 0 and world == 1:
+        if not args.no_extras:
+            extras = attn_extras(kd, torch, peaks, HN.L2Flush("cuda"))
+        if not args.no_cpu_baseline:
+            cpu = cpu_baseline(cfg, wl, host_steps[0])
+
+    if rank == 0:
+        achieved = flop_avg / attn_avg / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "traffic": None,
+                "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
+                "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                "kernel": "attn_tc_kernel (tree-verify attention)",
+                "algorithmic_flops_per_launch": flop_avg,
+                "algorithmic_bytes_per_launch": byte_avg,
+                "avg_launch_ms": round(attn_avg * 1e3, 4)}
+        line = {"metric": METRIC, "value": round(steps_per_s, 3), "unit": "verify steps/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(elapsed_max / args.steps * 1e3, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded N(0,1)/24 latents and queries, random trees, planted accepts)",
+                "config": {**config_json(cfg), "parallelism": f"replicas x{world} (requests per rank)"},
+                "attn_tflops": round(achieved, 2),
+                "attn_kv_hbm_gbs": round(byte_avg / attn_avg / 1e9, 1),
+                "attn_roofline_frac": round(max(flop_avg / (peaks["bf16_tflops"] * 1e12),
+                                                byte_avg / (peaks["hbm_gbs"] * 1e9)) / attn_avg, 4),
+                "attn_share_of_step": round(attn_avg / (elapsed / args.steps), 4),
+                "roofline": roof,
+                "e2e": {"value": round(e2e_rate, 3), "unit": "verify steps/s",
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "gpu_launches": V.launches_per_step * args.steps,
+                "clocks": clk.summary(),
+                "device_errors": err_bits}
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        if extras is not None:
+            line["per_config_attention"] = extras
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_kd(args)
+
+
+if __name__ == "__main__":
+    main()

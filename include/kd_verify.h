@@ -1,0 +1,205 @@
+/*
+ * kd_verify.h -- C ABI of libkdverify.so, the B200 (sm_100a) tree-verify step of
+ * DDTree speculative decoding for Multi-head Latent Attention (MLA) models.
+ *
+ * One verify step (sources are the pages' titles and sections):
+ *   1. kd_kv_write_nodes     the budget+1 node latents go to the next free slots,
+ *                            root first ("The Architectural Keystone: Writing the
+ *                            Model Header ...", "The Reasoning That Preceded the
+ *                            Header");
+ *   2. kd_tree_build_mask    per-node ancestor bitmasks from the parent array
+ *                            ("The Architecture of Pragmatic Ambition", "The
+ *                            Knowledge Architecture": attention over the tree with
+ *                            a visibility mask);
+ *   3. kd_tree_verify_attn   MLA attention in absorb form ("The Architecture of
+ *                            Pragmatic Ambition", "The Thinking Process") of every
+ *                            node and head over the committed cache and the node's
+ *                            tree ancestors;
+ *   4. kd_tree_accept        greedy walk to the longest path matching the target
+ *                            argmax ("The Knowledge Architecture");
+ *   5. kd_kv_compact         the accepted path's latents, root included, gathered
+ *                            into contiguous slots and the length advanced
+ *                            ("The Reasoning That Preceded the Header"; read-all-
+ *                            then-write, "Mistakes and Iterative Refinement").
+ *
+ * Conventions shared by every call
+ *   - All pointers except those documented as host pointers are DEVICE pointers on
+ *     the current CUDA device.  The caller allocates and owns every buffer,
+ *     workspace included; the library allocates nothing and keeps no state besides
+ *     cached device/function attributes.
+ *   - Every call is asynchronous on `stream`; results are valid after the stream
+ *     is synchronised.
+ *   - bf16 tensors are passed as kd_bf16_t (the 16-bit pattern of a bfloat16).
+ *   - Fixed MLA widths: latent d_c = 512, rope d_r = 64.  Limits: 1 <= n <= 128
+ *     tree nodes (budget <= 127), 1 <= H <= 128 heads, B >= 1.
+ *   - Request b's cache rows are c_kv[b*cap + j] (row stride kv_row_stride_c
+ *     elements) and k_rope[b*cap + j] (row stride kv_row_stride_r elements); a
+ *     576-wide interleaved layout is expressed by pointing k_rope at column 512
+ *     and passing stride 576 for both.
+ *   - Return value: KD_OK (0) or a negative KD_E* code.  Host-side validation
+ *     happens before anything is enqueued; a failing call enqueues nothing.
+ *   - Device-detected input errors (bad parent, cache overflow, bad accepted
+ *     length, ...) never trap: the kernel ORs a KD_DEV_* bit into the caller's
+ *     int32 device error word and treats the affected request as a no-op.  Read
+ *     it with kd_read_device_error().  For kd_tree_verify_attn the error word is
+ *     the first int32 of the workspace; the other calls take it as `dev_error`
+ *     (may be NULL, in which case device errors are only skipped).
+ */
+#ifndef KD_VERIFY_H
+#define KD_VERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t kd_bf16_t;
+
+/* return codes */
+#define KD_OK            0
+#define KD_EINVAL       -1   /* null pointer, bad shape/limit, misaligned pointer or stride */
+#define KD_ERANGE       -2   /* workspace too small / size beyond a documented maximum     */
+#define KD_ELAUNCH      -3   /* a CUDA call failed; kd_strerror() gives the CUDA text       */
+#define KD_ENODEV       -4   /* current device is not sm_100 (B200-class)                   */
+
+/* device error bits (ORed into the device error word) */
+#define KD_DEV_BAD_PARENT    0x01  /* parent[0] != -1 or parent[i] not in [0, i)       */
+#define KD_DEV_CACHE_FULL    0x02  /* cache_len + n (or + len) exceeds cap, or < 0     */
+#define KD_DEV_BAD_PATH      0x04  /* len not in [1, n] or path entry not in [0, n)     */
+#define KD_DEV_BAD_POSITION  0x08  /* positions[b][i] != cache_len[b] + depth(i)       */
+#define KD_DEV_TIMEOUT       0x10  /* a bounded wait inside a kernel gave up            */
+#define KD_DEV_BAD_MASK      0x20  /* a node's mask lacks bit 0 (root) or its own bit   */
+
+#define KD_D_C 512
+#define KD_D_R 64
+#define KD_MAX_NODES 128
+#define KD_MAX_HEADS 128
+
+/*
+ * kd_tree_build_mask -- ancestor bitmasks and depths of B trees.
+ *   parents [B][n] int32  topological: parents[b][0] == -1, 0 <= parents[b][i] < i.
+ *   vis     [B][n][W] uint32 out, W = (n+31)/32: bit k of word k/32 of row i is set
+ *           iff node k is node i or one of its ancestors.
+ *   depth   [B][n] int32 out (may be NULL): edges from the root.
+ *   A request with a bad parent array gets KD_DEV_BAD_PARENT and all-zero rows.
+ */
+int kd_tree_build_mask(const int32_t* parents, int B, int n, uint32_t* vis,
+                       int32_t* depth, int32_t* dev_error, cudaStream_t stream);
+
+/*
+ * kd_verify_workspace_bytes -- workspace size for kd_tree_verify_attn with the
+ * same B, n, H and kv_splits (0 = automatic).  Pure host arithmetic.  The
+ * workspace must be 256-byte aligned; its first int32 is the device error word,
+ * which the caller zeroes once (the library only ORs bits into it).
+ */
+size_t kd_verify_workspace_bytes(int B, int n, int H, int64_t cap, int kv_splits);
+
+/*
+ * kd_tree_verify_attn -- masked MLA-absorb attention of every tree node over its
+ * request's committed cache and its tree ancestors.
+ *
+ * For request b with L = cache_lens[b], node i, head h:
+ *   V(i)  = {0 .. L-1}  U  {L + k : bit k of vis[b][i] set}        (node k at slot L+k)
+ *   s_j   = scale * (q_nope_absorbed[b][i][h] . c_kv[j] + q_rope[b][i][h] . k_rope[j])
+ *   out[b][i][h] = sum_{j in V(i)} softmax(s)_j * c_kv[j]          (512-wide latent)
+ *   lse[b][i][h] = ln sum_{j in V(i)} exp(s_j)
+ *
+ *   q_nope_absorbed [B][n][H][512] bf16, contiguous (q_nope already multiplied by W_UK).
+ *   q_rope          [B][n][H][64]  bf16, contiguous, already rotated.
+ *   c_kv, k_rope    cache rows as described above, already holding the n node
+ *                   latents at slots L..L+n-1; rotated keys.  Base pointers and
+ *                   row strides must be 16-byte aligned (strides multiple of 8).
+ *   cap             slots per request; requires cache_lens[b] + n <= cap.
+ *   cache_lens [B]  int32 committed lengths (device).
+ *   vis [B][n][W]   uint32 node masks (e.g. from kd_tree_build_mask).
+ *   positions [B][n] int32 or NULL.  q_rope/k_rope arrive rotated, so positions do
+ *                   not enter the arithmetic; when given they are checked against
+ *                   cache_lens[b] + depth(i) and a mismatch sets KD_DEV_BAD_POSITION.
+ *   scale           softmax scale applied to the raw dot products.
+ *   out [B][n][H][512] bf16 out; lse [B][n][H] fp32 out (natural log; -inf if a
+ *                   node sees no key, which cannot happen with a valid mask).
+ *   workspace       >= kd_verify_workspace_bytes(B, n, H, cap, kv_splits) bytes.
+ *   kv_splits       0 = automatic; otherwise the number of key-range partitions
+ *                   per request (1 .. 64), combined by a log-sum-exp merge.
+ *   out/lse must not alias any input.
+ */
+int kd_tree_verify_attn(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* q_rope,
+                        const kd_bf16_t* c_kv, const kd_bf16_t* k_rope,
+                        int64_t kv_row_stride_c, int64_t kv_row_stride_r, int64_t cap,
+                        const int32_t* cache_lens, const uint32_t* vis,
+                        const int32_t* positions, int B, int n, int H, float scale,
+                        kd_bf16_t* out, float* lse, void* workspace, size_t ws_bytes,
+                        int kv_splits, cudaStream_t stream);
+
+/*
+ * kd_tree_verify_attn_simt -- the same operation as kd_tree_verify_attn computed on
+ * CUDA cores (one warp per node and head, keys streamed one at a time).  No
+ * workspace, no tensor cores; a plain second GPU implementation for bring-up and
+ * cross-checks.  Same arguments and checks; device errors go to `dev_error`
+ * (may be NULL).
+ */
+int kd_tree_verify_attn_simt(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* q_rope,
+                             const kd_bf16_t* c_kv, const kd_bf16_t* k_rope,
+                             int64_t kv_row_stride_c, int64_t kv_row_stride_r, int64_t cap,
+                             const int32_t* cache_lens, const uint32_t* vis,
+                             const int32_t* positions, int B, int n, int H, float scale,
+                             kd_bf16_t* out, float* lse, int32_t* dev_error,
+                             cudaStream_t stream);
+
+/*
+ * kd_tree_accept -- greedy acceptance of B verified trees.
+ *   node_tokens [B][n], parents [B][n], target_argmax [B][n] int32 (target_argmax[b][i]
+ *   is the target's prediction after node i).
+ *   Starting at the root, repeatedly step to the lowest-index child c of the current
+ *   node with node_tokens[c] == target_argmax[current]; stop when none matches.
+ *   path  [B][n] int32 out: path[b][0..len-1] = accepted nodes (path[b][0] = 0);
+ *                 entries from len on are set to -1.
+ *   len   [B]    int32 out: accepted count including the root (1 .. n).
+ *   bonus [B]    int32 out: target_argmax[b][last accepted node].
+ *   A bad parent array gives KD_DEV_BAD_PARENT and len = 1, path = {0}.
+ */
+int kd_tree_accept(const int32_t* node_tokens, const int32_t* parents,
+                   const int32_t* target_argmax, int B, int n, int32_t* path,
+                   int32_t* len, int32_t* bonus, int32_t* dev_error, cudaStream_t stream);
+
+/*
+ * kd_kv_compact -- gather each request's accepted latents into contiguous slots.
+ *   For j < len[b]: row L+j <- row L+path[b][j] of c_kv and k_rope (L = cache_lens[b]),
+ *   all rows read before any is written; then cache_lens[b] += len[b].  Rows below L
+ *   and from L+len on are untouched.  In place on c_kv, k_rope and cache_lens.
+ *   A request with len not in [1, n], a path entry not in [0, n) or L + n > cap is
+ *   left unchanged and sets KD_DEV_BAD_PATH / KD_DEV_CACHE_FULL.
+ */
+int kd_kv_compact(kd_bf16_t* c_kv, kd_bf16_t* k_rope, int64_t kv_row_stride_c,
+                  int64_t kv_row_stride_r, int64_t cap, const int32_t* path,
+                  const int32_t* len, int32_t* cache_lens, int B, int n,
+                  int32_t* dev_error, cudaStream_t stream);
+
+/*
+ * kd_kv_write_nodes -- store the n node latents of each request at slots L..L+n-1.
+ *   node_ckv [B][n][512], node_krope [B][n][64] bf16 contiguous.  cache_lens is not
+ *   changed.  A request with L + n > cap is skipped and sets KD_DEV_CACHE_FULL.
+ */
+int kd_kv_write_nodes(kd_bf16_t* c_kv, kd_bf16_t* k_rope, int64_t kv_row_stride_c,
+                      int64_t kv_row_stride_r, int64_t cap, const int32_t* cache_lens,
+                      const kd_bf16_t* node_ckv, const kd_bf16_t* node_krope, int B,
+                      int n, int32_t* dev_error, cudaStream_t stream);
+
+/*
+ * kd_read_device_error -- synchronises `stream`, returns the device error word
+ * (>= 0, KD_DEV_* bits) and zeroes it when `clear` is non-zero.  Negative return =
+ * KD_E* code of the copy itself.
+ */
+int kd_read_device_error(int32_t* dev_error, int clear, cudaStream_t stream);
+
+/* kd_strerror -- static text for a KD_E* code (KD_ELAUNCH: last CUDA error text). */
+const char* kd_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KD_VERIFY_H */

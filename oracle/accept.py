@@ -19,7 +19,7 @@ def tree_accept(node_tokens, parents, target_argmax):
     n = len(parents)
     path = [0]
     cur = 0
-    while True:
+    while len(path) < n:          # a root-to-node path has at most n nodes
         nxt = -1
         for c in range(n):
             if int(parents[c]) == cur and int(node_tokens[c]) == int(target_argmax[cur]):

@@ -1,0 +1,731 @@
+// Tree-verify MLA-absorb attention on sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Definition ("The Architecture of Pragmatic Ambition", "The Thinking Process" --
+// absorb form: q_nope . (W_UK c_kv) = (q_nope W_UK) . c_kv -- and "The Knowledge
+// Architecture" -- tree attention under a visibility mask; "The Architectural
+// Keystone ...", "The Reasoning That Preceded the Header" -- node k of the
+// budget+1 tree lives in slot L+k):
+//   row (i, h) of request b sees slots [0, L) and {L+k : bit k of vis[b][i]};
+//   s = scale (q_abs . c_kv + q_rope . k_rope), out = softmax(s) . c_kv, lse = ln sum exp s.
+//
+// Because the latent is shared by all heads, a request's n*H query rows against
+// its keys form a dense (n*H x 576) . (576 x keys) contraction followed by a
+// (n*H x keys) . (keys x 512) one.  Rows are node-major (row = i*H + h) and cut
+// into 128-row M tiles; keys are streamed in 128-key tiles.
+//
+// The fp32 output accumulator of one M tile (128 x 512) fills all 512 TMEM
+// columns of an SM, leaving none for scores, so each unit of work runs on a
+// 2-CTA cluster with split roles:
+//   rank 0 ("QK" CTA): Q tile resident in shared memory (9 x 16 KB TMA boxes,
+//       128-byte swizzle); a 4-stage ring of 128-key x 64-dim K chunks; S = Q K^T
+//       into a double-buffered 2 x 128-column TMEM accumulator; a 4-warp softmax
+//       group turns S into bf16 P (online max with a lazy rescale threshold) and
+//       stores P straight into rank 1's shared memory (st.shared::cluster) in the
+//       K-major 128-byte-swizzled layout the MMA reads.
+//   rank 1 ("PV" CTA): O (128 x 512 fp32) in TMEM; V chunks (128 keys x 64 latent
+//       columns, MN-major) in a 2-deep ring of 64 KB groups; O += P V as
+//       M=128, N=256, K=16 MMAs; a 4-warp group applies the rare O rescale and
+//       writes the normalised output (or a split-KV partial).
+// QK work (576-deep) and PV work (512-deep) are nearly equal, so the pair keeps
+// both tensor pipes busy.  The same c_kv tile is read by both CTAs (the second
+// read hits L2).  No TMA multicast is used anywhere.
+//
+// Every mbarrier wait is bounded (globaltimer); a wait that gives up raises
+// KD_DEV_TIMEOUT, marks both CTAs aborted, and every role falls through to the
+// common teardown (cluster barrier, TMEM release).
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "kd_common.cuh"
+#include "kd_ptx.cuh"
+
+namespace kd {
+
+int launch_combine(const float* part_o, const float* part_lse, const int32_t* cache_lens, int B,
+                   int n, int H, int64_t cap, int splits, uint16_t* out, float* lse,
+                   cudaStream_t stream);
+
+namespace tc {
+
+using namespace ptx;
+
+constexpr int BM = 128;                 // query rows per M tile
+constexpr int BN = 128;                 // keys per tile
+constexpr int KC = 64;                  // latent/rope columns per 128-byte swizzle atom
+constexpr int NCHUNK = 9;               // 8 latent chunks + 1 rope chunk
+constexpr int CHUNK = BN * KC * 2;      // 16 KB (also BM * KC * 2)
+constexpr int NK = 4;                   // K ring stages
+constexpr int VG = 4 * CHUNK;           // one V group: 128 keys x 256 latent columns
+constexpr int NVG = 2;                  // V ring depth
+constexpr int PSLOT = BM * BN * 2;      // one bf16 P tile (two 16 KB swizzle columns)
+
+// control block (same offsets in both CTAs so the peer can address it)
+constexpr int CTRL = 4096;
+enum Bar {
+  Q_FULL = 0,
+  K_FULL = 1,
+  K_EMPTY = K_FULL + NK,
+  S_FULL = K_EMPTY + NK,
+  S_EMPTY = S_FULL + 2,
+  P_FREE = S_EMPTY + 2,
+  V_FULL = P_FREE + 2,
+  V_EMPTY = V_FULL + NVG,
+  P_FULL = V_EMPTY + NVG,
+  PV_TILE = P_FULL + 2,
+  O_DONE = PV_TILE + 1,
+  EVENT = O_DONE + 1,
+  CORR_DONE = EVENT + 1,
+  STATS = CORR_DONE + 1,
+  DRAIN = STATS + 1,
+  NBAR = DRAIN + 1
+};
+constexpr int OFF_TMEM = 512;           // u32 TMEM base
+constexpr int OFF_ABORT = 516;          // u32 abort flag
+constexpr int OFF_EVTYPE = 520;         // u32 event type (1 rescale, 2 done)
+constexpr int OFF_EVTILE = 524;         // u32 P slot of a rescale event
+constexpr int OFF_FLAG = 528;           // u32 [2] rescale-needed flag per P slot
+constexpr int OFF_ALPHA = 1024;         // f32 [2][128] per-row rescale factor per P slot
+constexpr int OFF_MFIN = 2048;          // f32 [128] final running max (log2 units)
+constexpr int OFF_LFIN = 2560;          // f32 [128] final running sum
+static_assert(NBAR * 8 <= OFF_TMEM, "barrier block overflow");
+
+constexpr int Q_OFF = CTRL;
+constexpr int K_OFF = Q_OFF + NCHUNK * CHUNK;
+constexpr int QK_END = K_OFF + NK * CHUNK;
+constexpr int P_OFF = CTRL;
+constexpr int V_OFF = P_OFF + 2 * PSLOT;
+constexpr int PV_END = V_OFF + NVG * VG;
+constexpr int SMEM_BYTES = (QK_END > PV_END ? QK_END : PV_END) + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, 0, 0);    // Q, K both K-major
+constexpr uint32_t IDESC_PV = idesc_bf16(BM, 256, 0, 1);   // P K-major, V MN-major
+constexpr float RESCALE_THRESHOLD = 8.0f;                  // log2 units: P <= 2^8
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;          // 2 s per wait
+
+struct Params {
+  const int32_t* cache_lens;
+  const uint32_t* vis;
+  const int32_t* positions;
+  uint16_t* out;
+  float* lse;
+  float* part_o;
+  float* part_lse;
+  int32_t* err;
+  int64_t cap;
+  int B, n, H, W, mtiles, splits;
+  float scale_log2;
+};
+
+struct Ctx {
+  uint32_t base;          // shared address of the aligned block
+  volatile uint32_t* abort_flag;
+  uint32_t peer;          // cluster rank of the other CTA
+  int32_t* err;
+  __device__ uint32_t bar(int i) const { return base + 8u * (uint32_t)i; }
+};
+
+__device__ __noinline__ void abort_pair(const Ctx& cx) {
+  *cx.abort_flag = 1u;
+  st_cluster_u32(map_to_rank(cx.base + OFF_ABORT, cx.peer), 1u);
+  raise_dev_error(cx.err, KD_DEV_TIMEOUT);
+}
+
+// Bounded wait for the phase of `bar` with parity `par` to complete.
+__device__ __forceinline__ bool wait_bar(const Ctx& cx, uint32_t bar, uint32_t par,
+                                         bool cluster_scope = false) {
+  if (cluster_scope ? mbar_try_wait_cluster(bar, par) : mbar_try_wait(bar, par)) return true;
+  uint64_t t0 = 0;
+  for (uint32_t spin = 1;; ++spin) {
+    if (cluster_scope ? mbar_try_wait_cluster(bar, par) : mbar_try_wait(bar, par)) return true;
+    if ((spin & 63u) == 0u) {
+      if (*cx.abort_flag) return false;
+      const uint64_t t = globaltimer();
+      if (t0 == 0) t0 = t;
+      else if (t - t0 > WAIT_LIMIT_NS) { abort_pair(cx); return false; }
+    }
+  }
+}
+
+// Warp-uniform outcome of a wait (all 32 lanes call it).
+__device__ __forceinline__ bool wait_warp(const Ctx& cx, uint32_t bar, uint32_t par,
+                                          bool cluster_scope = false) {
+  return __all_sync(0xffffffffu, wait_bar(cx, bar, par, cluster_scope));
+}
+
+// Group-uniform outcome of a wait for a 128-thread group sharing named barrier `id`.
+__device__ __forceinline__ bool wait_group(const Ctx& cx, uint32_t bar, uint32_t par, uint32_t id,
+                                           bool cluster_scope = false) {
+  const bool ok = wait_bar(cx, bar, par, cluster_scope);
+  return !named_bar_red_or(id, 128, !ok);
+}
+
+__device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {      // K-major, SW128
+  return smem_desc_sw128(saddr, 16, 1024);
+}
+__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) {     // MN-major, SW128, 16 KB atoms
+  return smem_desc_sw128(saddr, CHUNK, 1024);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant__ CUtensorMap tm_qr,
+               const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
+               const __grid_constant__ Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+
+  const uint32_t rank = cluster_ctarank();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int unit = (int)cluster_id_x();
+  const int mt = unit % p.mtiles;
+  const int sp = (unit / p.mtiles) % p.splits;
+  const int b = unit / (p.mtiles * p.splits);
+  const int n = p.n, H = p.H;
+
+  const int64_t L = p.cache_lens[b];
+  if (L < 0 || L + n > p.cap) {          // both CTAs see the same value and leave together
+    if (rank == 0 && threadIdx.x == 0 && mt == 0 && sp == 0) raise_dev_error(p.err, KD_DEV_CACHE_FULL);
+    return;
+  }
+  const int64_t nkeys = L + n;
+  const int T = (int)((nkeys + BN - 1) / BN);
+  const int t0 = (int)((int64_t)sp * T / p.splits), t1 = (int)((int64_t)(sp + 1) * T / p.splits);
+  const int ntiles = t1 - t0;
+  const int64_t kbeg = (int64_t)t0 * BN;                    // request-relative first key
+  const int64_t krow0 = (int64_t)b * p.cap + kbeg;          // cache row of the first key
+  const int rows_req = n * H;
+  const int qrow0 = b * rows_req + mt * BM;
+
+  Ctx cx;
+  cx.base = base;
+  cx.abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + OFF_ABORT);
+  cx.peer = rank ^ 1u;
+  cx.err = p.err;
+
+  if (threadIdx.x == 0) {
+    const uint32_t counts[NBAR] = {
+        1,                   // Q_FULL
+        1, 1, 1, 1,          // K_FULL
+        1, 1, 1, 1,          // K_EMPTY
+        1, 1,                // S_FULL
+        128, 128,            // S_EMPTY
+        1, 1,                // P_FREE
+        1, 1,                // V_FULL
+        1, 1,                // V_EMPTY
+        1, 1,                // P_FULL
+        1,                   // PV_TILE
+        1,                   // O_DONE
+        1,                   // EVENT
+        128,                 // CORR_DONE
+        1,                   // STATS
+        1};                  // DRAIN
+    static_assert(sizeof(counts) / sizeof(counts[0]) == NBAR, "barrier counts");
+    for (int i = 0; i < NBAR; ++i) mbar_init(cx.bar(i), counts[i]);
+    *cx.abort_flag = 0u;
+    fence_mbar_init();
+  }
+  const uint32_t tmem_cols = rank == 0 ? 256u : 512u;
+  if (warp == 1) {
+    tmem_alloc(base + OFF_TMEM, tmem_cols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_qa);
+    tma_prefetch_desc(&tm_qr);
+    tma_prefetch_desc(&tm_c);
+    tma_prefetch_desc(&tm_r);
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + OFF_TMEM);
+
+  if (rank == 0) {
+    // ======================================================= QK CTA
+    if (warp == 0) {
+      // ---------------- TMA producer: Q once, then K chunks
+      if (lane == 0 && ntiles > 0) {
+        bool ok = true;
+        mbar_arrive_expect_tx(cx.bar(Q_FULL), NCHUNK * CHUNK);
+        for (int c = 0; c < 8; ++c)
+          tma_load_2d(base + Q_OFF + c * CHUNK, &tm_qa, c * KC, qrow0, cx.bar(Q_FULL));
+        tma_load_2d(base + Q_OFF + 8 * CHUNK, &tm_qr, 0, qrow0, cx.bar(Q_FULL));
+        uint32_t it = 0;
+        for (int t = 0; t < ntiles && ok; ++t) {
+          const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN);
+          for (int c = 0; c < NCHUNK; ++c, ++it) {
+            const uint32_t st = it % NK, k = it / NK;
+            if (!(ok = wait_bar(cx, cx.bar(K_EMPTY + st), (k & 1u) ^ 1u))) break;
+            mbar_arrive_expect_tx(cx.bar(K_FULL + st), CHUNK);
+            if (c < 8) tma_load_2d(base + K_OFF + st * CHUNK, &tm_c, c * KC, krow, cx.bar(K_FULL + st));
+            else tma_load_2d(base + K_OFF + st * CHUNK, &tm_r, 0, krow, cx.bar(K_FULL + st));
+          }
+        }
+        // drain: every armed stage must have landed before the CTA can exit
+        wait_bar(cx, cx.bar(Q_FULL), 0);
+        for (uint32_t j = (it > NK ? it - NK : 0); j < it; ++j)
+          wait_bar(cx, cx.bar(K_FULL + j % NK), (j / NK) & 1u);
+      }
+    } else if (warp == 1) {
+      // ---------------- MMA issuer: S[sb] = Q K^T
+      if (lane == 0 && ntiles > 0) {
+        bool ok = wait_bar(cx, cx.bar(Q_FULL), 0);
+        tc_fence_after();
+        uint32_t it = 0;
+        for (int t = 0; t < ntiles && ok; ++t) {
+          const uint32_t sb = t & 1;
+          if (!(ok = wait_bar(cx, cx.bar(S_EMPTY + sb), ((t >> 1) & 1) ^ 1))) break;
+          tc_fence_after();
+          const uint32_t d = tmem + sb * BN;
+          for (int c = 0; c < NCHUNK; ++c, ++it) {
+            const uint32_t st = it % NK;
+            if (!(ok = wait_bar(cx, cx.bar(K_FULL + st), (it / NK) & 1u))) break;
+            tc_fence_after();
+            const uint32_t a0 = base + Q_OFF + c * CHUNK, b0 = base + K_OFF + st * CHUNK;
+#pragma unroll
+            for (int kk = 0; kk < KC / 16; ++kk)
+              mma_bf16_ss(d, desc_k(a0 + kk * 32), desc_k(b0 + kk * 32), IDESC_QK, (c | kk) != 0);
+            tc_commit(cx.bar(K_EMPTY + st));
+          }
+          if (ok) tc_commit(cx.bar(S_FULL + sb));
+        }
+        tc_commit(cx.bar(DRAIN));
+        wait_bar(cx, cx.bar(DRAIN), 0);
+      }
+      __syncwarp();
+    } else {
+      // ---------------- softmax group (warps 2..5): one thread per query row
+      const int quad = warp & 3;
+      const int r = quad * 32 + lane;
+      const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+      const int R = mt * BM + r;
+      const bool valid = R < rows_req;
+      const int node = valid ? R / H : 0;
+      const int W = p.W;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      for (int q = 0; q < W; ++q) w[q] = p.vis[((size_t)b * n + node) * W + q];
+      if (valid && sp == 0 && (R % H) == 0) {
+        int depth = -1;
+        for (int q = 0; q < W; ++q) depth += __popc(w[q]);
+        if (!(w[0] & 1u) || !((w[node >> 5] >> (node & 31)) & 1u)) raise_dev_error(p.err, KD_DEV_BAD_MASK);
+        if (p.positions && p.positions[(size_t)b * n + node] != (int32_t)(L + depth))
+          raise_dev_error(p.err, KD_DEV_BAD_POSITION);
+      }
+      const uint32_t peer_p = map_to_rank(base + P_OFF, cx.peer);
+      const uint32_t peer_ctrl = map_to_rank(base, cx.peer);
+      float m_ref = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int t = 0; t < ntiles && ok; ++t) {
+        const uint32_t sb = t & 1;
+        if (!(ok = wait_group(cx, cx.bar(S_FULL + sb), (t >> 1) & 1, 1))) break;
+        tc_fence_after();
+        float x[BN];
+        {
+          uint32_t v[32];
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            tmem_ld32(lane_addr + sb * BN + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(v[k]) * p.scale_log2;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(cx.bar(S_EMPTY + sb));
+        // mask: only keys at or beyond L need it
+        const int64_t kt = kbeg + (int64_t)t * BN;
+        if (kt + BN > L) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c) {
+            const int64_t k = kt + c - L;
+            bool vis_c = true;
+            if (k >= 0) vis_c = (k < n) && ((w[(int)k >> 5] >> ((int)k & 31)) & 1u);
+            if (!vis_c) x[c] = -INFINITY;
+          }
+        }
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) tmax = fmaxf(tmax, x[c]);
+        float alpha = 1.f;
+        bool rescale_row = false;
+        if (tmax > m_ref + RESCALE_THRESHOLD) {
+          if (m_ref != -INFINITY) {
+            alpha = ex2(m_ref - tmax);
+            rescale_row = true;
+          } else {
+            alpha = 0.f;
+          }
+          l *= alpha;
+          m_ref = tmax;
+        }
+        const float mb = m_ref == -INFINITY ? 0.f : m_ref;
+        float rs = 0.f;
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int c = 0; c < BN / 2; ++c) {
+          const float p0 = ex2(x[2 * c] - mb), p1 = ex2(x[2 * c + 1] - mb);
+          rs += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        l += rs;
+        // P slot sb is free once the PV MMAs of tile t-2 completed
+        if (!(ok = wait_group(cx, cx.bar(P_FREE + sb), ((t >> 1) & 1) ^ 1, 1))) break;
+        const uint32_t prow = peer_p + sb * PSLOT + (uint32_t)r * 128u;
+#pragma unroll
+        for (int q = 0; q < BN / 8; ++q) {
+          const uint32_t atom = q >> 3, chunk = (q & 7) ^ (r & 7);
+          st_cluster_v4(prow + atom * (BM * 128) + chunk * 16, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
+                        pk[4 * q + 3]);
+        }
+        st_cluster_u32(peer_ctrl + OFF_ALPHA + (sb * BM + r) * 4, __float_as_uint(alpha));
+        fence_proxy_async_cluster();
+        const bool any = named_bar_red_or(1, 128, rescale_row);
+        if (r == 0) {
+          st_cluster_u32(peer_ctrl + OFF_FLAG + sb * 4, any ? 1u : 0u);
+          mbar_arrive_remote(peer_ctrl + 8u * P_FULL + 8u * sb);
+        }
+      }
+      // final row statistics for the epilogue
+      st_cluster_u32(peer_ctrl + OFF_MFIN + r * 4, __float_as_uint(m_ref));
+      st_cluster_u32(peer_ctrl + OFF_LFIN + r * 4, __float_as_uint(l));
+      named_bar_sync(1, 128);
+      if (r == 0) mbar_arrive_remote(peer_ctrl + 8u * STATS);
+      // the last P_FREE arrivals come from the peer's MMA completion: wait for them
+      if (ok && r == 0)
+        for (int t = (ntiles > 2 ? ntiles - 2 : 0); t < ntiles; ++t)
+          wait_bar(cx, cx.bar(P_FREE + (t & 1)), (t >> 1) & 1);
+    }
+  } else {
+    // ======================================================= PV CTA
+    if (warp == 0) {
+      // ---------------- TMA producer: V groups (128 keys x 256 latent columns)
+      if (lane == 0) {
+        bool ok = true;
+        uint32_t gi = 0;
+        for (int t = 0; t < ntiles && ok; ++t) {
+          const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN);
+          for (int hh = 0; hh < 2; ++hh, ++gi) {
+            const uint32_t g = gi % NVG, k = gi / NVG;
+            if (!(ok = wait_bar(cx, cx.bar(V_EMPTY + g), (k & 1u) ^ 1u))) break;
+            mbar_arrive_expect_tx(cx.bar(V_FULL + g), VG);
+            for (int q = 0; q < 4; ++q)
+              tma_load_2d(base + V_OFF + g * VG + q * CHUNK, &tm_c, (hh * 4 + q) * KC, krow,
+                          cx.bar(V_FULL + g));
+          }
+        }
+        for (uint32_t j = (gi > NVG ? gi - NVG : 0); j < gi; ++j)
+          wait_bar(cx, cx.bar(V_FULL + j % NVG), (j / NVG) & 1u);
+      }
+    } else if (warp == 1) {
+      // ---------------- MMA issuer: O += P V
+      volatile uint32_t* ctrl = reinterpret_cast<volatile uint32_t*>(gbase);
+      bool ok = true;
+      uint32_t gi = 0, nres = 0;
+      for (int t = 0; t < ntiles && ok; ++t) {
+        const uint32_t sb = t & 1;
+        if (!(ok = wait_warp(cx, cx.bar(P_FULL + sb), (t >> 1) & 1, true))) break;
+        fence_proxy_async_cta();
+        const uint32_t flag = ctrl[(OFF_FLAG >> 2) + sb];
+        if (flag && t > 0) {
+          // every earlier PV MMA must be done before O is rescaled
+          if (!(ok = wait_warp(cx, cx.bar(PV_TILE), (t - 1) & 1))) break;
+          if (lane == 0) {
+            ctrl[OFF_EVTYPE >> 2] = 1u;
+            ctrl[OFF_EVTILE >> 2] = sb;
+            mbar_arrive(cx.bar(EVENT));
+          }
+          if (!(ok = wait_warp(cx, cx.bar(CORR_DONE), nres & 1u))) break;
+          ++nres;
+        }
+        tc_fence_after();
+        const int64_t kt = kbeg + (int64_t)t * BN;
+        const int nvalid = (int)((nkeys - kt) < BN ? (nkeys - kt) : BN);
+        for (int hh = 0; hh < 2 && ok; ++hh, ++gi) {
+          const uint32_t g = gi % NVG;
+          if (!(ok = wait_warp(cx, cx.bar(V_FULL + g), (gi / NVG) & 1u))) break;
+          if (nvalid < BN) {
+            // rows past the request's last key may hold anything (even NaN bit
+            // patterns); P is 0 there but 0 * NaN is not, so clear them
+            uint4* vg = reinterpret_cast<uint4*>(gbase + V_OFF + g * VG);
+            const int per_chunk = (BN - nvalid) * 8;
+            for (int idx = lane; idx < 4 * per_chunk; idx += 32) {
+              const int q = idx / per_chunk, e = idx % per_chunk;
+              vg[q * (CHUNK / 16) + nvalid * 8 + e] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_cta();
+            __syncwarp();
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t pa = base + P_OFF + sb * PSLOT, vb = base + V_OFF + g * VG;
+#pragma unroll
+            for (int ks = 0; ks < BN / 16; ++ks)
+              mma_bf16_ss(tmem + hh * 256, desc_k(pa + (ks >> 2) * (BM * 128) + (ks & 3) * 32),
+                          desc_mn(vb + ks * 2048), IDESC_PV, (t > 0 || ks > 0) ? 1u : 0u);
+            tc_commit(cx.bar(V_EMPTY + g));
+          }
+          __syncwarp();
+        }
+        if (ok && lane == 0) {
+          tc_commit(cx.bar(PV_TILE));
+          tc_commit_mc(cx.bar(P_FREE + sb), (uint16_t)(1u << cx.peer));
+        }
+        __syncwarp();
+      }
+      if (lane == 0) {
+        if (ntiles > 0) tc_commit(cx.bar(O_DONE));
+        else mbar_arrive(cx.bar(O_DONE));
+        ctrl[OFF_EVTYPE >> 2] = 2u;
+        mbar_arrive(cx.bar(EVENT));
+      }
+      __syncwarp();
+    } else {
+      // ---------------- correction / epilogue group (warps 2..5)
+      volatile uint32_t* ctrl = reinterpret_cast<volatile uint32_t*>(gbase);
+      const volatile float* fctrl = reinterpret_cast<const volatile float*>(gbase);
+      const int quad = warp & 3;
+      const int r = quad * 32 + lane;
+      const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+      bool ok = true;
+      uint32_t nev = 0;
+      while (true) {
+        if (!(ok = wait_group(cx, cx.bar(EVENT), nev & 1u, 1))) break;
+        ++nev;
+        if (ctrl[OFF_EVTYPE >> 2] != 1u) break;
+        const uint32_t sb = ctrl[OFF_EVTILE >> 2];
+        const float a = fctrl[(OFF_ALPHA >> 2) + sb * BM + r];
+        tc_fence_after();
+        uint32_t v[32];
+        for (int c = 0; c < 512 / 32; ++c) {
+          tmem_ld32(lane_addr + c * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * a);
+          tmem_st32(lane_addr + c * 32, v);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(cx.bar(CORR_DONE));
+      }
+      if (ok) ok = wait_group(cx, cx.bar(STATS), 0, 1, true);
+      if (ok) ok = wait_group(cx, cx.bar(O_DONE), 0, 1);
+      tc_fence_after();
+      const float m = ok ? fctrl[(OFF_MFIN >> 2) + r] : 0.f;
+      const float l = ok ? fctrl[(OFF_LFIN >> 2) + r] : 0.f;
+      const int R = mt * BM + r;
+      const bool valid = ok && R < rows_req;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const bool have_o = ntiles > 0;
+      const int64_t grow = (int64_t)b * rows_req + R;
+      const int64_t prow = ((int64_t)sp * p.B * rows_req) + grow;
+      uint32_t v[32];
+      for (int c = 0; c < 512 / 32; ++c) {
+        if (have_o && ok) {
+          tmem_ld32(lane_addr + c * 32, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] = 0u;
+        }
+        if (!valid) continue;
+        if (p.splits == 1) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + grow * KD_D_C + c * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t a0 = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
+            uint32_t a1 = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
+            uint32_t a2 = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
+            uint32_t a3 = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
+            dst[q] = make_uint4(a0, a1, a2, a3);
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.part_o + prow * KD_D_C + c * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(v[4 * q]) * inv, __uint_as_float(v[4 * q + 1]) * inv,
+                                 __uint_as_float(v[4 * q + 2]) * inv, __uint_as_float(v[4 * q + 3]) * inv);
+        }
+      }
+      if (valid) {
+        const float lse_v = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (p.splits == 1) p.lse[grow] = lse_v;
+        else p.part_lse[prow] = lse_v;
+      }
+      tc_fence_before();
+    }
+  }
+
+  // ------------------------------------------------------- teardown
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// 2-D bf16 view [rows][inner] with `row_bytes` pitch, 64 x 128 boxes, 128-byte swizzle.
+static int make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint64_t row_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return KD_ELAUNCH;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {KC, 128};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+    return KD_ELAUNCH;
+  }
+  return KD_OK;
+}
+
+// Co-resident 2-CTA clusters of the kernel on the current device (cached).
+static int active_pairs(int sms) {
+  static int cached[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  int pairs = sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeClusterDimension;
+  at.val.clusterDim.x = 2;
+  at.val.clusterDim.y = 1;
+  at.val.clusterDim.z = 1;
+  cfg.attrs = &at;
+  cfg.numAttrs = 1;
+  int nc = 0;
+  if (cudaOccupancyMaxActiveClusters(&nc, attn_tc_kernel, &cfg) == cudaSuccess && nc > 0) pairs = nc;
+  cudaGetLastError();
+  if (dev >= 0 && dev < 64) cached[dev] = pairs;
+  return pairs;
+}
+
+}  // namespace tc
+
+// Split count for B requests of n nodes and H heads when the caller leaves it to
+// the library: minimise waves x (tiles per unit + fixed cost) over the pairs that
+// fit at once, with key length bounded by cap.
+int auto_splits(int B, int n, int H, int64_t cap, int pairs) {
+  const int64_t mtiles = ((int64_t)n * H + tc::BM - 1) / tc::BM;
+  const int64_t units = (int64_t)B * mtiles;
+  const int64_t T = (cap + tc::BN - 1) / tc::BN;
+  int best = 1;
+  double best_cost = 1e300;
+  for (int s = 1; s <= 64 && s <= T; ++s) {
+    const int64_t waves = (units * s + pairs - 1) / pairs;
+    const double cost = (double)waves * ((double)((T + s - 1) / s) + 2.0) + (s > 1 ? 1.0 : 0.0);
+    if (cost < best_cost * 0.98) { best_cost = cost; best = s; }
+  }
+  return best;
+}
+
+size_t workspace_bytes_for(int B, int n, int H, int splits) {
+  size_t bytes = 256;
+  if (splits > 1) {
+    const size_t rows = (size_t)B * n * H;
+    bytes += ((rows * splits * 4 + 255) / 256) * 256;       // partial lse
+    bytes += rows * splits * KD_D_C * 4;                     // partial out
+  }
+  return bytes;
+}
+
+}  // namespace kd
+
+using namespace kd;
+
+extern "C" size_t kd_verify_workspace_bytes(int B, int n, int H, int64_t cap, int kv_splits) {
+  if (!shapes_ok(B, n) || H < 1 || H > KD_MAX_HEADS || cap < 1 || kv_splits < 0 || kv_splits > 64) return 0;
+  const int s = kv_splits > 0 ? kv_splits : auto_splits(B, n, H, cap, 74);
+  return workspace_bytes_for(B, n, H, s);
+}
+
+extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_rope,
+                                   const kd_bf16_t* c_kv, const kd_bf16_t* k_rope, int64_t sc,
+                                   int64_t sr, int64_t cap, const int32_t* cache_lens,
+                                   const uint32_t* vis, const int32_t* positions, int B, int n,
+                                   int H, float scale, kd_bf16_t* out, float* lse, void* workspace,
+                                   size_t ws_bytes, int kv_splits, cudaStream_t stream) {
+  if (!q_abs || !q_rope || !cache_lens || !vis || !out || !lse || !workspace ||
+      !shapes_ok(B, n) || H < 1 || H > KD_MAX_HEADS || !cache_ok(c_kv, k_rope, sc, sr, cap) ||
+      !aligned16(q_abs) || !aligned16(q_rope) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) || !(scale > 0.f) || kv_splits < 0 ||
+      kv_splits > 64)
+    return KD_EINVAL;
+  const int64_t rows = (int64_t)B * n * H;
+  if (rows > INT32_MAX || (int64_t)B * cap > INT32_MAX) return KD_EINVAL;
+  int sms = 0;
+  int st = device_sms(&sms);
+  if (st) return st;
+  static bool attr_set[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    st = cuda_status(cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          tc::SMEM_BYTES),
+                     "cudaFuncSetAttribute(attn_tc_kernel)");
+    if (st) return st;
+    attr_set[dev] = true;
+  }
+  int splits = kv_splits;
+  if (splits == 0) {
+    splits = auto_splits(B, n, H, cap, tc::active_pairs(sms));
+    while (splits > 1 && workspace_bytes_for(B, n, H, splits) > ws_bytes) --splits;
+  }
+  if (workspace_bytes_for(B, n, H, splits) > ws_bytes) return KD_ERANGE;
+
+  CUtensorMap tq, tr, tcv, tkr;
+  if ((st = tc::make_map(&tq, q_abs, KD_D_C, (uint64_t)rows, KD_D_C * 2))) return st;
+  if ((st = tc::make_map(&tr, q_rope, KD_D_R, (uint64_t)rows, KD_D_R * 2))) return st;
+  if ((st = tc::make_map(&tcv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2))) return st;
+  if ((st = tc::make_map(&tkr, k_rope, KD_D_R, (uint64_t)(B * cap), (uint64_t)sr * 2))) return st;
+
+  tc::Params prm;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  prm.cache_lens = cache_lens;
+  prm.vis = vis;
+  prm.positions = positions;
+  prm.out = out;
+  prm.lse = lse;
+  prm.err = reinterpret_cast<int32_t*>(ws);
+  prm.part_lse = splits > 1 ? reinterpret_cast<float*>(ws + 256) : nullptr;
+  prm.part_o = splits > 1 ? reinterpret_cast<float*>(ws + 256 + ((rows * splits * 4 + 255) / 256) * 256)
+                          : nullptr;
+  prm.cap = cap;
+  prm.B = B;
+  prm.n = n;
+  prm.H = H;
+  prm.W = (n + 31) / 32;
+  prm.mtiles = (int)((rows / B + tc::BM - 1) / tc::BM);
+  prm.splits = splits;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  const int64_t units = (int64_t)B * prm.mtiles * splits;
+  if (2 * units > INT32_MAX) return KD_EINVAL;
+  tc::attn_tc_kernel<<<dim3((unsigned)(2 * units)), 192, tc::SMEM_BYTES, stream>>>(tq, tr, tcv, tkr, prm);
+  st = launch_status("attn_tc_kernel");
+  if (st || splits == 1) return st;
+  return launch_combine(prm.part_o, prm.part_lse, cache_lens, B, n, H, cap, splits, out, lse, stream);
+}

@@ -1,0 +1,302 @@
+// Tree and cache kernels of the verify step: ancestor masks, greedy acceptance,
+// node-latent write and post-accept compaction.  All are launch-latency-sized;
+// they are written for coalesced 16-byte traffic and warp-level decisions.
+//
+// Sources (page title, section):
+//   "The Architecture of Pragmatic Ambition" -- "The Knowledge Architecture":
+//       visibility-masked tree attention; greedy walk to the longest prefix that
+//       matches the target's predictions.
+//   "The Architectural Keystone: Writing the Model Header ..." -- "The Reasoning
+//       That Preceded the Header": budget+1 nodes, root at the next free slot,
+//       accepted latents (root included) gathered into contiguous slots and the
+//       cache length advanced by the accepted count; "Mistakes and Iterative
+//       Refinement": source and destination slots of the gather can overlap, so
+//       every kept row is read before any is written.
+
+#include <string.h>
+
+#include "kd_common.cuh"
+
+namespace kd {
+
+// ------------------------------------------------------------------ host helpers
+static thread_local char g_cuda_err[256];
+
+void set_cuda_error(cudaError_t e, const char* where) {
+  snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", where, cudaGetErrorString(e));
+}
+
+int device_sms(int* sms) {
+  static int cached_major[64], cached_sms[64];
+  int dev = 0;
+  int st = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st) return st;
+  if (dev < 0 || dev >= 64) return KD_ENODEV;
+  if (cached_major[dev] == 0) {
+    int major = 0, count = 0;
+    st = cuda_status(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "attr");
+    if (st) return st;
+    st = cuda_status(cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev), "attr");
+    if (st) return st;
+    cached_sms[dev] = count;
+    cached_major[dev] = major;
+  }
+  if (cached_major[dev] != 10) return KD_ENODEV;
+  if (sms) *sms = cached_sms[dev];
+  return KD_OK;
+}
+
+// ------------------------------------------------------------------ mask build
+// One CTA per request, one thread per node.  A node's mask is the OR of the bits
+// of the nodes met walking parent links from it to the root.
+__global__ void __launch_bounds__(KD_MAX_NODES)
+build_mask_kernel(const int32_t* __restrict__ parents, int n, uint32_t* __restrict__ vis,
+                  int32_t* __restrict__ depth, int32_t* dev_error) {
+  __shared__ int par[KD_MAX_NODES];
+  const int b = blockIdx.x, i = threadIdx.x;
+  const int W = (n + 31) >> 5;
+  int p = 0;
+  bool bad = false;
+  if (i < n) {
+    p = parents[(size_t)b * n + i];
+    bad = (i == 0) ? (p != -1) : (p < 0 || p >= i);
+    par[i] = p;
+  }
+  bad = __syncthreads_or(bad);
+  if (i >= n) return;
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  int d = 0;
+  if (!bad) {
+    int k = i;
+    while (k > 0) {             // parent < child, so at most i steps
+      w[k >> 5] |= 1u << (k & 31);
+      k = par[k];
+      ++d;
+    }
+    w[0] |= 1u;                 // the root is visible to every node
+  } else if (i == 0) {
+    raise_dev_error(dev_error, KD_DEV_BAD_PARENT);
+  }
+  uint32_t* row = vis + ((size_t)b * n + i) * W;
+  for (int q = 0; q < W; ++q) row[q] = w[q];
+  if (depth) depth[(size_t)b * n + i] = d;
+}
+
+// ------------------------------------------------------------------ greedy accept
+// One warp per request.  Lane l holds nodes l, l+32, l+64, l+96.  Each step is
+// one ballot per 32-node chunk; the first chunk with a match gives the
+// lowest-index matching child.
+__global__ void __launch_bounds__(128)
+accept_kernel(const int32_t* __restrict__ tokens, const int32_t* __restrict__ parents,
+              const int32_t* __restrict__ argmax, int B, int n, int32_t* __restrict__ path,
+              int32_t* __restrict__ len, int32_t* __restrict__ bonus, int32_t* dev_error) {
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (b >= B) return;
+  const size_t base = (size_t)b * n;
+  int par[4], tok[4];
+  bool bad = false;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int node = c * 32 + lane;
+    par[c] = -2;
+    tok[c] = 0;
+    if (node < n) {
+      par[c] = parents[base + node];
+      tok[c] = tokens[base + node];
+      bad |= (node == 0) ? (par[c] != -1) : (par[c] < 0 || par[c] >= node);
+    }
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  int cur = 0, cnt = 1;
+  if (lane == 0) path[base] = 0;
+  if (bad) {
+    if (lane == 0) raise_dev_error(dev_error, KD_DEV_BAD_PARENT);
+  } else {
+    while (cnt < n) {
+      const int want = argmax[base + cur];
+      int next = -1;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const unsigned m = __ballot_sync(0xffffffffu, par[c] == cur && tok[c] == want);
+        if (next < 0 && m) next = c * 32 + __ffs(m) - 1;
+      }
+      if (next < 0) break;
+      cur = next;
+      if (lane == 0) path[base + cnt] = cur;
+      ++cnt;
+    }
+  }
+  for (int j = cnt + lane; j < n; j += 32) path[base + j] = -1;
+  if (lane == 0) {
+    len[b] = cnt;
+    bonus[b] = argmax[base + cur];
+  }
+}
+
+// ------------------------------------------------------------------ node write
+// One CTA per request; 16-byte copies of the n node rows into slots L..L+n-1.
+__global__ void __launch_bounds__(256)
+write_nodes_kernel(uint4* __restrict__ c_kv, uint4* __restrict__ k_rope, int64_t sc16,
+                   int64_t sr16, int64_t cap, const int32_t* __restrict__ cache_lens,
+                   const uint4* __restrict__ node_ckv, const uint4* __restrict__ node_krope,
+                   int n, int32_t* dev_error) {
+  const int b = blockIdx.x;
+  const int64_t L = cache_lens[b];
+  if (L < 0 || L + n > cap) {
+    if (threadIdx.x == 0) raise_dev_error(dev_error, KD_DEV_CACHE_FULL);
+    return;
+  }
+  constexpr int CC = KD_D_C / 8, CR = KD_D_R / 8;   // uint4 per row
+  const int64_t row0 = (int64_t)b * cap + L;
+  for (int idx = threadIdx.x; idx < n * (CC + CR); idx += blockDim.x) {
+    const int k = idx / (CC + CR), q = idx % (CC + CR);
+    if (q < CC)
+      c_kv[(row0 + k) * sc16 + q] = node_ckv[((size_t)b * n + k) * CC + q];
+    else
+      k_rope[(row0 + k) * sr16 + (q - CC)] = node_krope[((size_t)b * n + k) * CR + (q - CC)];
+  }
+}
+
+// ------------------------------------------------------------------ compaction
+// One CTA per request.  Phase 1 reads every row that moves (path[j] != j) into
+// shared memory; phase 2 writes them to slots L+j.  Rows with path[j] == j are
+// already in place.  Shared memory holds up to n rows of 1152 bytes.
+__global__ void __launch_bounds__(256)
+compact_kernel(uint4* __restrict__ c_kv, uint4* __restrict__ k_rope, int64_t sc16, int64_t sr16,
+               int64_t cap, const int32_t* __restrict__ path, const int32_t* __restrict__ len,
+               int32_t* __restrict__ cache_lens, int n, int32_t* dev_error) {
+  extern __shared__ uint4 stage[];
+  __shared__ int src[KD_MAX_NODES], dst[KD_MAX_NODES];
+  __shared__ int moves, ok;
+  constexpr int CC = KD_D_C / 8, CR = KD_D_R / 8, ROW = CC + CR;
+  const int b = blockIdx.x;
+  const int64_t L = cache_lens[b];
+  const int m = len[b];
+  if (threadIdx.x == 0) {
+    int good = 1, err = 0;
+    if (m < 1 || m > n) { good = 0; err |= KD_DEV_BAD_PATH; }
+    if (L < 0 || L + n > cap) { good = 0; err |= KD_DEV_CACHE_FULL; }
+    int c = 0;
+    for (int j = 0; good && j < m; ++j) {
+      const int p = path[(size_t)b * n + j];
+      if (p < 0 || p >= n) { good = 0; err |= KD_DEV_BAD_PATH; break; }
+      if (p != j) { src[c] = p; dst[c] = j; ++c; }
+    }
+    moves = c;
+    ok = good;
+    if (err) raise_dev_error(dev_error, err);
+  }
+  __syncthreads();
+  if (!ok) return;
+  const int64_t row0 = (int64_t)b * cap + L;
+  const int total = moves * ROW;
+  for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {      // read all ...
+    const int r = idx / ROW, q = idx % ROW;
+    const int64_t s = row0 + src[r];
+    stage[idx] = (q < CC) ? c_kv[s * sc16 + q] : k_rope[s * sr16 + (q - CC)];
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {      // ... then write
+    const int r = idx / ROW, q = idx % ROW;
+    const int64_t d = row0 + dst[r];
+    if (q < CC) c_kv[d * sc16 + q] = stage[idx];
+    else k_rope[d * sr16 + (q - CC)] = stage[idx];
+  }
+  if (threadIdx.x == 0) cache_lens[b] = (int32_t)(L + m);
+}
+
+}  // namespace kd
+
+using namespace kd;
+
+// ================================================================== C ABI
+extern "C" int kd_tree_build_mask(const int32_t* parents, int B, int n, uint32_t* vis,
+                                  int32_t* depth, int32_t* dev_error, cudaStream_t stream) {
+  if (!parents || !vis || !shapes_ok(B, n)) return KD_EINVAL;
+  int st = device_sms(nullptr);
+  if (st) return st;
+  build_mask_kernel<<<B, KD_MAX_NODES, 0, stream>>>(parents, n, vis, depth, dev_error);
+  return launch_status("build_mask_kernel");
+}
+
+extern "C" int kd_tree_accept(const int32_t* node_tokens, const int32_t* parents,
+                              const int32_t* target_argmax, int B, int n, int32_t* path,
+                              int32_t* len, int32_t* bonus, int32_t* dev_error,
+                              cudaStream_t stream) {
+  if (!node_tokens || !parents || !target_argmax || !path || !len || !bonus || !shapes_ok(B, n))
+    return KD_EINVAL;
+  int st = device_sms(nullptr);
+  if (st) return st;
+  const int per_cta = 4;
+  accept_kernel<<<(B + per_cta - 1) / per_cta, 32 * per_cta, 0, stream>>>(
+      node_tokens, parents, target_argmax, B, n, path, len, bonus, dev_error);
+  return launch_status("accept_kernel");
+}
+
+extern "C" int kd_kv_write_nodes(kd_bf16_t* c_kv, kd_bf16_t* k_rope, int64_t sc, int64_t sr,
+                                 int64_t cap, const int32_t* cache_lens, const kd_bf16_t* node_ckv,
+                                 const kd_bf16_t* node_krope, int B, int n, int32_t* dev_error,
+                                 cudaStream_t stream) {
+  if (!cache_ok(c_kv, k_rope, sc, sr, cap) || !cache_lens || !node_ckv || !node_krope ||
+      !aligned16(node_ckv) || !aligned16(node_krope) || !shapes_ok(B, n))
+    return KD_EINVAL;
+  int st = device_sms(nullptr);
+  if (st) return st;
+  write_nodes_kernel<<<B, 256, 0, stream>>>(
+      reinterpret_cast<uint4*>(c_kv), reinterpret_cast<uint4*>(k_rope), sc / 8, sr / 8, cap,
+      cache_lens, reinterpret_cast<const uint4*>(node_ckv),
+      reinterpret_cast<const uint4*>(node_krope), n, dev_error);
+  return launch_status("write_nodes_kernel");
+}
+
+extern "C" int kd_kv_compact(kd_bf16_t* c_kv, kd_bf16_t* k_rope, int64_t sc, int64_t sr,
+                             int64_t cap, const int32_t* path, const int32_t* len,
+                             int32_t* cache_lens, int B, int n, int32_t* dev_error,
+                             cudaStream_t stream) {
+  if (!cache_ok(c_kv, k_rope, sc, sr, cap) || !path || !len || !cache_lens || !shapes_ok(B, n))
+    return KD_EINVAL;
+  int st = device_sms(nullptr);
+  if (st) return st;
+  const size_t smem = (size_t)n * (KD_D_C + KD_D_R) * 2;
+  static bool attr_set[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    st = cuda_status(cudaFuncSetAttribute(compact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          KD_MAX_NODES * (KD_D_C + KD_D_R) * 2),
+                     "cudaFuncSetAttribute(compact_kernel)");
+    if (st) return st;
+    attr_set[dev] = true;
+  }
+  compact_kernel<<<B, 256, smem, stream>>>(reinterpret_cast<uint4*>(c_kv),
+                                           reinterpret_cast<uint4*>(k_rope), sc / 8, sr / 8, cap,
+                                           path, len, cache_lens, n, dev_error);
+  return launch_status("compact_kernel");
+}
+
+extern "C" int kd_read_device_error(int32_t* dev_error, int clear, cudaStream_t stream) {
+  if (!dev_error) return KD_EINVAL;
+  int32_t v = 0;
+  int st = cuda_status(cudaMemcpyAsync(&v, dev_error, sizeof(v), cudaMemcpyDeviceToHost, stream),
+                       "cudaMemcpyAsync(error word)");
+  if (st) return st;
+  if (clear) {
+    st = cuda_status(cudaMemsetAsync(dev_error, 0, sizeof(int32_t), stream), "cudaMemsetAsync");
+    if (st) return st;
+  }
+  st = cuda_status(cudaStreamSynchronize(stream), "cudaStreamSynchronize");
+  if (st) return st;
+  return v;
+}
+
+extern "C" const char* kd_strerror(int code) {
+  switch (code) {
+    case KD_OK: return "ok";
+    case KD_EINVAL: return "invalid argument (null pointer, shape, limit or alignment)";
+    case KD_ERANGE: return "workspace too small or size beyond the supported maximum";
+    case KD_ELAUNCH: return g_cuda_err[0] ? g_cuda_err : "CUDA error";
+    case KD_ENODEV: return "current device is not an sm_100 (B200-class) GPU";
+    default: return "unknown kd error code";
+  }
+}

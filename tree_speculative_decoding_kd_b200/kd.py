@@ -1,0 +1,231 @@
+"""ctypes binding of libkdverify.so (declared in include/kd_verify.h).
+
+Argument marshalling only: shape/dtype checks, ``data_ptr()``s, the current
+CUDA stream.  Every step of the verify path runs in the library's kernels.
+Importing this module raises if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkdverify.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m tree_speculative_decoding_kd_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_i64 = ctypes.c_int64
+_f = ctypes.c_float
+_sz = ctypes.c_size_t
+
+_SIGS = {
+    "kd_tree_build_mask": (_i, [_p, _i, _i, _p, _p, _p, _p]),
+    "kd_verify_workspace_bytes": (_sz, [_i, _i, _i, _i64, _i]),
+    "kd_tree_verify_attn": (_i, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i, _f,
+                                 _p, _p, _p, _sz, _i, _p]),
+    "kd_tree_verify_attn_simt": (_i, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i,
+                                      _f, _p, _p, _p, _p]),
+    "kd_tree_accept": (_i, [_p, _p, _p, _i, _i, _p, _p, _p, _p, _p]),
+    "kd_kv_compact": (_i, [_p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _p, _p]),
+    "kd_kv_write_nodes": (_i, [_p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _p, _p]),
+    "kd_read_device_error": (_i, [_p, _i, _p]),
+    "kd_strerror": (ctypes.c_char_p, [_i]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+D_C, D_R = 512, 64
+KD_DEV_BITS = {0x01: "BAD_PARENT", 0x02: "CACHE_FULL", 0x04: "BAD_PATH",
+               0x08: "BAD_POSITION", 0x10: "TIMEOUT", 0x20: "BAD_MASK"}
+
+
+class KdError(RuntimeError):
+    pass
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise KdError(f"{what}: {lib.kd_strerror(rc).decode()} (code {rc})")
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t, dtype, name, contiguous=True):
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    dts = dtype if isinstance(dtype, tuple) else (dtype,)
+    if t.dtype not in dts:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dts}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _cache_strides(c_kv, k_rope):
+    """Row strides (elements) of [B][cap][512] / [B][cap][64] cache views."""
+    _need(c_kv, torch.bfloat16, "c_kv", contiguous=False)
+    _need(k_rope, torch.bfloat16, "k_rope", contiguous=False)
+    B, cap, dc = c_kv.shape
+    if dc != D_C or tuple(k_rope.shape) != (B, cap, D_R):
+        raise ValueError("c_kv must be [B][cap][512] and k_rope [B][cap][64]")
+    for t in (c_kv, k_rope):
+        if t.stride(2) != 1 or t.stride(0) != cap * t.stride(1):
+            raise ValueError("cache rows must be unit-stride with uniform row pitch")
+    return c_kv.stride(1), k_rope.stride(1), cap
+
+
+def new_error_word(device=None) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def kd_tree_build_mask(parents, vis=None, depth=None, dev_error=None, stream=None):
+    _need(parents, torch.int32, "parents")
+    B, n = parents.shape
+    W = (n + 31) // 32
+    if vis is None:
+        vis = torch.empty(B, n, W, dtype=torch.int32, device=parents.device)
+    if depth is None:
+        depth = torch.empty(B, n, dtype=torch.int32, device=parents.device)
+    _check(lib.kd_tree_build_mask(_ptr(parents), B, n, _ptr(vis), _ptr(depth), _ptr(dev_error),
+                                  _stream(stream)), "kd_tree_build_mask")
+    return vis, depth
+
+
+def kd_verify_workspace_bytes(B, n, H, cap, kv_splits=0) -> int:
+    return int(lib.kd_verify_workspace_bytes(B, n, H, cap, kv_splits))
+
+
+def new_workspace(B, n, H, cap, kv_splits=0, device=None) -> torch.Tensor:
+    """Zeroed workspace (its first int32 is the device error word)."""
+    nbytes = kd_verify_workspace_bytes(B, n, H, cap, kv_splits)
+    if nbytes == 0:
+        raise ValueError("invalid shape for the verify workspace")
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def _attn_args(q_abs, q_rope, c_kv, k_rope, cache_lens, vis, positions, out, lse):
+    _need(q_abs, torch.bfloat16, "q_abs")
+    _need(q_rope, torch.bfloat16, "q_rope")
+    _need(cache_lens, torch.int32, "cache_lens")
+    _need(vis, (torch.int32, torch.uint32), "vis")
+    B, n, H, dc = q_abs.shape
+    if dc != D_C or tuple(q_rope.shape) != (B, n, H, D_R):
+        raise ValueError("q_abs must be [B][n][H][512] and q_rope [B][n][H][64]")
+    if positions is not None:
+        _need(positions, torch.int32, "positions")
+    sc, sr, cap = _cache_strides(c_kv, k_rope)
+    if out is None:
+        out = torch.empty(B, n, H, D_C, dtype=torch.bfloat16, device=q_abs.device)
+    if lse is None:
+        lse = torch.empty(B, n, H, dtype=torch.float32, device=q_abs.device)
+    _need(out, torch.bfloat16, "out")
+    _need(lse, torch.float32, "lse")
+    return B, n, H, sc, sr, cap, out, lse
+
+
+def kd_tree_verify_attn(q_abs, q_rope, c_kv, k_rope, cache_lens, vis, positions=None,
+                        scale=1.0 / math.sqrt(192.0), out=None, lse=None, workspace=None,
+                        kv_splits=0, stream=None):
+    B, n, H, sc, sr, cap, out, lse = _attn_args(q_abs, q_rope, c_kv, k_rope, cache_lens, vis,
+                                                positions, out, lse)
+    if workspace is None:
+        workspace = new_workspace(B, n, H, cap, kv_splits, q_abs.device)
+    _check(lib.kd_tree_verify_attn(_ptr(q_abs), _ptr(q_rope), _ptr(c_kv), _ptr(k_rope), sc, sr,
+                                   cap, _ptr(cache_lens), _ptr(vis), _ptr(positions), B, n, H,
+                                   float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), int(kv_splits),
+                                   _stream(stream)), "kd_tree_verify_attn")
+    return out, lse
+
+
+def kd_tree_verify_attn_simt(q_abs, q_rope, c_kv, k_rope, cache_lens, vis, positions=None,
+                             scale=1.0 / math.sqrt(192.0), out=None, lse=None, dev_error=None,
+                             stream=None):
+    B, n, H, sc, sr, cap, out, lse = _attn_args(q_abs, q_rope, c_kv, k_rope, cache_lens, vis,
+                                                positions, out, lse)
+    _check(lib.kd_tree_verify_attn_simt(_ptr(q_abs), _ptr(q_rope), _ptr(c_kv), _ptr(k_rope), sc,
+                                        sr, cap, _ptr(cache_lens), _ptr(vis), _ptr(positions), B,
+                                        n, H, float(scale), _ptr(out), _ptr(lse),
+                                        _ptr(dev_error), _stream(stream)),
+           "kd_tree_verify_attn_simt")
+    return out, lse
+
+
+def kd_tree_accept(node_tokens, parents, target_argmax, path=None, length=None, bonus=None,
+                   dev_error=None, stream=None):
+    for t, nm in ((node_tokens, "node_tokens"), (parents, "parents"), (target_argmax, "target_argmax")):
+        _need(t, torch.int32, nm)
+    B, n = parents.shape
+    dev = parents.device
+    path = torch.empty(B, n, dtype=torch.int32, device=dev) if path is None else path
+    length = torch.empty(B, dtype=torch.int32, device=dev) if length is None else length
+    bonus = torch.empty(B, dtype=torch.int32, device=dev) if bonus is None else bonus
+    _check(lib.kd_tree_accept(_ptr(node_tokens), _ptr(parents), _ptr(target_argmax), B, n,
+                              _ptr(path), _ptr(length), _ptr(bonus), _ptr(dev_error),
+                              _stream(stream)), "kd_tree_accept")
+    return path, length, bonus
+
+
+def kd_kv_compact(c_kv, k_rope, path, length, cache_lens, dev_error=None, stream=None):
+    sc, sr, cap = _cache_strides(c_kv, k_rope)
+    _need(path, torch.int32, "path")
+    _need(length, torch.int32, "len")
+    _need(cache_lens, torch.int32, "cache_lens")
+    B, n = path.shape
+    _check(lib.kd_kv_compact(_ptr(c_kv), _ptr(k_rope), sc, sr, cap, _ptr(path), _ptr(length),
+                             _ptr(cache_lens), B, n, _ptr(dev_error), _stream(stream)),
+           "kd_kv_compact")
+
+
+def kd_kv_write_nodes(c_kv, k_rope, cache_lens, node_ckv, node_krope, dev_error=None, stream=None):
+    sc, sr, cap = _cache_strides(c_kv, k_rope)
+    _need(node_ckv, torch.bfloat16, "node_ckv")
+    _need(node_krope, torch.bfloat16, "node_krope")
+    _need(cache_lens, torch.int32, "cache_lens")
+    B, n, _ = node_ckv.shape
+    _check(lib.kd_kv_write_nodes(_ptr(c_kv), _ptr(k_rope), sc, sr, cap, _ptr(cache_lens),
+                                 _ptr(node_ckv), _ptr(node_krope), B, n, _ptr(dev_error),
+                                 _stream(stream)), "kd_kv_write_nodes")
+
+
+def kd_read_device_error(word, clear=True, stream=None) -> int:
+    """Device error bits from an error word or a verify workspace (its first int32)."""
+    rc = lib.kd_read_device_error(_ptr(word), int(bool(clear)), _stream(stream))
+    if rc < 0:
+        _check(rc, "kd_read_device_error")
+    return rc
+
+
+def decode_device_error(bits: int) -> list:
+    return [name for bit, name in KD_DEV_BITS.items() if bits & bit]
+
+
+# ------------------------------------------------------------------ host <-> device helpers
+def bf16_from_bits(u16, device="cuda") -> torch.Tensor:
+    """numpy uint16 bf16 bit patterns -> bf16 tensor on ``device``."""
+    import numpy as np
+    t = torch.from_numpy(np.ascontiguousarray(u16).view(np.int16))
+    return t.to(device).view(torch.bfloat16)
+
+
+def bits_from_bf16(t: torch.Tensor):
+    """bf16 tensor -> numpy uint16 bit patterns (on the host)."""
+    import numpy as np
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
