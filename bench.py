@@ -41,6 +41,9 @@ def parse():
     ap.add_argument("--impl", choices=["kd", "reference"], default="kd")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-config attention lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--attn-only", default=None, choices=["tiny", "kimi_single", "batched", "long"],
+                    help="time only the attention of one single-step configuration")
+    ap.add_argument("--reps", type=int, default=20)
     return ap.parse_args()
 
 
@@ -189,44 +192,62 @@ class Verifier:
         kd.kd_kv_compact(self.c_kv, self.k_rope, self.path, self.len, self.lens, self.err)
 
 
+def attn_case(kd, torch, peaks, flush, name, reps=20, warm=3):
+    """Attention-only timing of one single-step configuration (L2 flushed per rep)."""
+    wl = W.make_workload(name)
+    cfg, st = wl.cfg, wl.step
+    qa, qr = kd.bf16_from_bits(st.q_abs), kd.bf16_from_bits(st.q_rope)
+    ck, kr = kd.bf16_from_bits(wl.c_kv), kd.bf16_from_bits(wl.k_rope)
+    lens = torch.from_numpy(wl.cache_lens.astype(np.int32)).cuda()
+    parents = torch.from_numpy(st.parents).cuda()
+    vis, _ = kd.kd_tree_build_mask(parents)
+    ws = kd.new_workspace(cfg.B, cfg.n, cfg.H, cfg.cap)
+    out = torch.empty(cfg.B, cfg.n, cfg.H, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(cfg.B, cfg.n, cfg.H, dtype=torch.float32, device="cuda")
+
+    def call():
+        kd.kd_tree_verify_attn(qa, qr, ck, kr, lens, vis, None, cfg.scale, out, lse, ws)
+
+    for _ in range(warm):
+        call()
+    times = []
+    for _ in range(reps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3)
+    bits = kd.kd_read_device_error(ws)
+    t = float(np.median(times))
+    depths = [_depths(p) for p in st.parents]
+    fl = HN.attn_flops(wl.cache_lens, depths, cfg.H)
+    by = HN.attn_bytes(wl.cache_lens, cfg.n, cfg.H)
+    t_fl, t_by = fl / (peaks["bf16_tflops"] * 1e12), by / (peaks["hbm_gbs"] * 1e9)
+    res = {"us": round(t * 1e6, 2), "us_min": round(min(times) * 1e6, 2),
+           "tflops": round(fl / t / 1e12, 1), "hbm_gbs": round(by / t / 1e9, 1),
+           "roofline_frac": round(max(t_fl, t_by) / t, 3), "bound": "tensor" if t_fl > t_by else "hbm",
+           "splits": "auto", "l2": "flushed (256 MB write) before each rep", "device_errors": bits}
+    del qa, qr, ck, kr, ws, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def attn_extras(kd, torch, peaks, flush):
     """Attention-only timings of the single-step configurations (parity cases)."""
-    res = {}
-    for name in ["tiny", "kimi_single", "batched", "long"]:
-        wl = W.make_workload(name)
-        cfg, st = wl.cfg, wl.step
-        qa, qr = kd.bf16_from_bits(st.q_abs), kd.bf16_from_bits(st.q_rope)
-        ck, kr = kd.bf16_from_bits(wl.c_kv), kd.bf16_from_bits(wl.k_rope)
-        lens = torch.from_numpy(wl.cache_lens.astype(np.int32)).cuda()
-        parents = torch.from_numpy(st.parents).cuda()
-        vis, _ = kd.kd_tree_build_mask(parents)
-        ws = kd.new_workspace(cfg.B, cfg.n, cfg.H, cfg.cap)
-        out = torch.empty(cfg.B, cfg.n, cfg.H, 512, dtype=torch.bfloat16, device="cuda")
-        lse = torch.empty(cfg.B, cfg.n, cfg.H, dtype=torch.float32, device="cuda")
-        call = lambda: kd.kd_tree_verify_attn(qa, qr, ck, kr, lens, vis, None, cfg.scale, out, lse, ws)  # noqa: E731
-        for _ in range(3):
-            call()
-        times = []
-        for _ in range(20):
-            flush()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            call()
-            e1.record()
-            torch.cuda.synchronize()
-            times.append(e0.elapsed_time(e1) * 1e-3)
-        t = float(np.median(times))
-        depths = [_depths(p) for p in st.parents]
-        fl = HN.attn_flops(wl.cache_lens, depths, cfg.H)
-        by = HN.attn_bytes(wl.cache_lens, cfg.n, cfg.H)
-        roof_t = max(fl / (peaks["bf16_tflops"] * 1e12), by / (peaks["hbm_gbs"] * 1e9))
-        res[name] = {"us": round(t * 1e6, 2), "tflops": round(fl / t / 1e12, 1),
-                     "hbm_gbs": round(by / t / 1e9, 1), "roofline_frac": round(roof_t / t, 3),
-                     "bound": "tensor" if fl / (peaks["bf16_tflops"] * 1e12) > by / (peaks["hbm_gbs"] * 1e9) else "hbm",
-                     "l2": "flushed (256 MB write) before each rep"}
-        del qa, qr, ck, kr, ws, out
-        torch.cuda.empty_cache()
-    return res
+    return {name: attn_case(kd, torch, peaks, flush, name) for name in
+            ["tiny", "kimi_single", "batched", "long"]}
+
+
+def run_attn_only(args):
+    """--attn-only NAME: time just the attention of one configuration (profiling aid)."""
+    import torch
+    torch.cuda.set_device(0)
+    from tree_speculative_decoding_kd_b200 import kd
+    peaks = HN.load_peaks(ROOT)
+    res = attn_case(kd, torch, peaks, HN.L2Flush("cuda"), args.attn_only, reps=args.reps, warm=1)
+    print(json.dumps({"attn_only": args.attn_only, **res}), flush=True)
 
 
 def run_kd(args):
@@ -371,7 +392,9 @@ def run_kd(args):
 
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.attn_only:
+        run_attn_only(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_kd(args)

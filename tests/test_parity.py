@@ -142,7 +142,8 @@ def test_accept_budget0_and_max_nodes(kd):
         tokens = np.stack([W.draw_tokens(rng, p) for p in parents])
         argmax = np.zeros_like(tokens)
         argmax[:, :-1] = tokens[:, 1:]          # every chain fully accepted
-        argmax[2, 5] = (tokens[2, 6] + 1) % W.VOCAB
+        if n > 6:
+            argmax[2, 5] = (tokens[2, 6] + 1) % W.VOCAB     # third chain stops after node 5
         path, ln, bonus = kd.kd_tree_accept(dev_i32(tokens), dev_i32(parents), dev_i32(argmax))
         torch.cuda.synchronize()
         rp, rl, rb = tree_accept_batch(tokens, parents, argmax)
@@ -372,3 +373,62 @@ def test_verify_loop_steps_match_oracle(kd):
         assert np.array_equal(host_u16(kd, kr), r_np)
     assert kd.kd_read_device_error(err) == 0
     assert kd.kd_read_device_error(ws) == 0
+
+
+# ------------------------------------------------------------------ full sizes, sampled rows
+def _sample_nodes(cfg, rng, per_req=3):
+    nodes = []
+    for b in range(cfg.B):
+        pick = {0, cfg.n - 1, int(rng.integers(1, cfg.n))} if cfg.n > 1 else {0}
+        nodes += [(b, i) for i in sorted(pick)][:per_req]
+    return nodes
+
+
+@pytest.mark.parametrize("name", ["batched", "long"])
+def test_attn_full_size_sampled(kd, name):
+    """Configs 3 and 4 at full size with automatic splitting (the bench's launch
+    configuration); the oracle computes three nodes of every request."""
+    wl = W.make_workload(name)
+    out, lse, bits = run_attn(kd, wl)
+    nodes = _sample_nodes(wl.cfg, np.random.default_rng(5))
+    ro, rl = oracle_attn(wl, nodes=nodes)
+    assert bits == 0
+    assert np.isfinite(out).all()
+    assert_attn(out, lse, ro, rl, f"{name} full")
+
+
+def test_loop_full_size_two_steps(kd):
+    """Config 5 exactly (64 requests, cap 18101): two whole steps, caches and
+    lengths bit-exact, attention on sampled nodes."""
+    cfg = W.CONFIGS["loop"]
+    wl = W.make_loop_state(cfg)
+    c_np, r_np, lens_np = wl.c_kv, wl.k_rope, wl.cache_lens.copy()
+    ck, kr, lens = dev_bf16(kd, c_np), dev_bf16(kd, r_np), dev_i32(lens_np)
+    err = kd.new_error_word()
+    ws = kd.new_workspace(cfg.B, cfg.n, cfg.H, cfg.cap)
+    rng = np.random.default_rng(6)
+    for s in range(2):
+        st = W.draw_step(cfg, s, with_nodes=True)
+        kd.kd_kv_write_nodes(ck, kr, lens, dev_bf16(kd, st.node_ckv), dev_bf16(kd, st.node_krope), err)
+        vis, depth = kd.kd_tree_build_mask(dev_i32(st.parents), dev_error=err)
+        pos = lens[:, None] + depth
+        out, lse = kd.kd_tree_verify_attn(dev_bf16(kd, st.q_abs), dev_bf16(kd, st.q_rope), ck, kr,
+                                          lens, vis, pos, cfg.scale, workspace=ws)
+        path, ln, bonus = kd.kd_tree_accept(dev_i32(st.tokens), dev_i32(st.parents),
+                                            dev_i32(st.argmax), dev_error=err)
+        kd.kd_kv_compact(ck, kr, path, ln, lens, err)
+        torch.cuda.synchronize()
+        res = oracle.verify_step(c_np, r_np, lens_np, st.parents, st.tokens, st.argmax, st.q_abs,
+                                 st.q_rope, cfg.scale, st.node_ckv, st.node_krope,
+                                 attn_nodes=_sample_nodes(cfg, rng, 2))
+        o = kd.bits_from_bf16(out)
+        assert_attn((o.astype(np.uint32) << 16).view(np.float32), lse.cpu().numpy(), res["out"],
+                    res["lse"], f"loop step {s}")
+        assert np.array_equal(path.cpu().numpy(), res["path"])
+        assert np.array_equal(ln.cpu().numpy(), res["len"])
+        assert np.array_equal(bonus.cpu().numpy(), res["bonus"])
+        c_np, r_np, lens_np = res["c_kv"], res["k_rope"], res["cache_lens"]
+        assert np.array_equal(lens.cpu().numpy(), lens_np)
+        assert np.array_equal(host_u16(kd, ck), c_np)
+        assert np.array_equal(host_u16(kd, kr), r_np)
+    assert kd.kd_read_device_error(err) == 0 and kd.kd_read_device_error(ws) == 0
