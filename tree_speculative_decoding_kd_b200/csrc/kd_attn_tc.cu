@@ -16,19 +16,22 @@
 // The fp32 output accumulator of one M tile (128 x 512) fills all 512 TMEM
 // columns of an SM, leaving none for scores, so each unit of work runs on a
 // 2-CTA cluster with split roles:
-//   rank 0 ("QK" CTA): Q tile resident in shared memory (9 x 16 KB TMA boxes,
-//       128-byte swizzle); a 4-stage ring of 128-key x 64-dim K chunks; S = Q K^T
-//       into a double-buffered 2 x 128-column TMEM accumulator; a 4-warp softmax
-//       group turns S into bf16 P (online max with a lazy rescale threshold) and
-//       stores P straight into rank 1's shared memory (st.shared::cluster) in the
-//       K-major 128-byte-swizzled layout the MMA reads.
-//   rank 1 ("PV" CTA): O (128 x 512 fp32) in TMEM; V chunks (128 keys x 64 latent
-//       columns, MN-major) in a 2-deep ring of 64 KB groups; O += P V as
-//       M=128, N=256, K=16 MMAs; a 4-warp group applies the rare O rescale and
-//       writes the normalised output (or a split-KV partial).
+//   rank 0 ("QK" CTA): S = Q K^T into a double-buffered 2 x 128-column TMEM
+//       accumulator.  Seven of Q's nine 64-wide chunks sit in TMEM and feed the MMA
+//       as its A operand from tensor memory; the other two sit in shared memory.
+//       That leaves shared memory for an 11-stage ring of 128-key x 64-column K
+//       chunks (TMA, 128-byte swizzle), enough lead time to hide L2/HBM latency.
+//       Two 4-warp softmax groups split each S tile's columns, keep an online max
+//       with a lazy rescale threshold, and store bf16 P straight into rank 1's
+//       shared memory (st.shared::cluster) in the K-major swizzled layout the MMA
+//       reads.
+//   rank 1 ("PV" CTA): O (128 x 512 fp32) in TMEM; V as 64-key x 256-column
+//       groups (four 64-column MN-major boxes) in a 4-deep ring; O += P V as
+//       M=128, N=256, K=16 MMAs; two 4-warp groups apply the rare O rescale and
+//       write the normalised output (or a split-KV partial), 256 columns each.
 // QK work (576-deep) and PV work (512-deep) are nearly equal, so the pair keeps
-// both tensor pipes busy.  The same c_kv tile is read by both CTAs (the second
-// read hits L2).  No TMA multicast is used anywhere.
+// both tensor pipes busy.  Both CTAs read the same c_kv tile (the second read
+// hits L2).  No TMA multicast is used anywhere.
 //
 // Every mbarrier wait is bounded (globaltimer); a wait that gives up raises
 // KD_DEV_TIMEOUT, marks both CTAs aborted, and every role falls through to the
@@ -51,21 +54,31 @@ namespace tc {
 
 using namespace ptx;
 
+constexpr int NTHREADS = 320;           // warp 0 TMA, warp 1 MMA, warps 2..9 two 4-warp groups
+constexpr int GROUP = 256;              // threads of the two 4-warp groups
 constexpr int BM = 128;                 // query rows per M tile
 constexpr int BN = 128;                 // keys per tile
-constexpr int KC = 64;                  // latent/rope columns per 128-byte swizzle atom
+constexpr int KC = 64;                  // columns per 128-byte swizzle atom
 constexpr int NCHUNK = 9;               // 8 latent chunks + 1 rope chunk
-constexpr int CHUNK = BN * KC * 2;      // 16 KB (also BM * KC * 2)
-constexpr int NK = 4;                   // K ring stages
-constexpr int VG = 4 * CHUNK;           // one V group: 128 keys x 256 latent columns
-constexpr int NVG = 2;                  // V ring depth
+constexpr int CHUNK = BN * KC * 2;      // 16 KB: 128 rows x 64 bf16
+constexpr int NQT = 7;                  // Q chunks held in TMEM (the rest in shared memory)
+constexpr int NK = 11;                  // K ring stages
+constexpr int VKEYS = 64;               // keys per V group
+constexpr int VCH = VKEYS * KC * 2;     // 8 KB: 64 keys x 64 latent columns
+constexpr int VG = 4 * VCH;             // one V group: 64 keys x 256 latent columns
+constexpr int NVG = 4;                  // V ring depth
 constexpr int PSLOT = BM * BN * 2;      // one bf16 P tile (two 16 KB swizzle columns)
+
+// TMEM columns of the QK CTA
+constexpr uint32_t TS = 0;              // S[2]: 2 x 128 columns
+constexpr uint32_t TQ = 256;            // Q chunks 0..6: 7 x 32 columns
 
 // control block (same offsets in both CTAs so the peer can address it)
 constexpr int CTRL = 4096;
 enum Bar {
   Q_FULL = 0,
-  K_FULL = 1,
+  QT_FULL = Q_FULL + 1,
+  K_FULL = QT_FULL + 1,
   K_EMPTY = K_FULL + NK,
   S_FULL = K_EMPTY + NK,
   S_EMPTY = S_FULL + 2,
@@ -83,16 +96,17 @@ enum Bar {
 };
 constexpr int OFF_TMEM = 512;           // u32 TMEM base
 constexpr int OFF_ABORT = 516;          // u32 abort flag
-constexpr int OFF_EVTYPE = 520;         // u32 event type (1 rescale, 2 done)
-constexpr int OFF_EVTILE = 524;         // u32 P slot of a rescale event
-constexpr int OFF_FLAG = 528;           // u32 [2] rescale-needed flag per P slot
-constexpr int OFF_ALPHA = 1024;         // f32 [2][128] per-row rescale factor per P slot
-constexpr int OFF_MFIN = 2048;          // f32 [128] final running max (log2 units)
-constexpr int OFF_LFIN = 2560;          // f32 [128] final running sum
+constexpr int OFF_EVTYPE = 520;         // u32 event type (1 rescale, 2 done)     [PV]
+constexpr int OFF_EVTILE = 524;         // u32 P slot of a rescale event           [PV]
+constexpr int OFF_FLAG = 528;           // u32 [2] rescale-needed flag per P slot  [PV, remote]
+constexpr int OFF_ALPHA = 1024;         // f32 [2][128] per-row rescale factor     [PV, remote]
+constexpr int OFF_MFIN = 2048;          // f32 [128] final running max (log2)      [PV, remote]
+constexpr int OFF_LFIN = 2560;          // f32 [128] final running sum             [PV, remote]
+constexpr int OFF_XCH = 3072;           // f32 [2][128] max / sum exchange         [QK, local]
 static_assert(NBAR * 8 <= OFF_TMEM, "barrier block overflow");
 
-constexpr int Q_OFF = CTRL;
-constexpr int K_OFF = Q_OFF + NCHUNK * CHUNK;
+constexpr int Q_OFF = CTRL;                           // Q chunks 7, 8
+constexpr int K_OFF = Q_OFF + (NCHUNK - NQT) * CHUNK;
 constexpr int QK_END = K_OFF + NK * CHUNK;
 constexpr int P_OFF = CTRL;
 constexpr int V_OFF = P_OFF + 2 * PSLOT;
@@ -109,6 +123,7 @@ struct Params {
   const int32_t* cache_lens;
   const uint32_t* vis;
   const int32_t* positions;
+  const uint16_t* q_abs;
   uint16_t* out;
   float* lse;
   float* part_o;
@@ -155,24 +170,414 @@ __device__ __forceinline__ bool wait_warp(const Ctx& cx, uint32_t bar, uint32_t 
   return __all_sync(0xffffffffu, wait_bar(cx, bar, par, cluster_scope));
 }
 
-// Group-uniform outcome of a wait for a 128-thread group sharing named barrier `id`.
-__device__ __forceinline__ bool wait_group(const Ctx& cx, uint32_t bar, uint32_t par, uint32_t id,
+// Group-uniform outcome of a wait for the 256-thread group at named barrier 1.
+__device__ __forceinline__ bool wait_group(const Ctx& cx, uint32_t bar, uint32_t par,
                                            bool cluster_scope = false) {
   const bool ok = wait_bar(cx, bar, par, cluster_scope);
-  return !named_bar_red_or(id, 128, !ok);
+  return !named_bar_red_or(1, GROUP, !ok);
 }
 
 __device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {      // K-major, SW128
   return smem_desc_sw128(saddr, 16, 1024);
 }
-__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) {     // MN-major, SW128, 16 KB atoms
-  return smem_desc_sw128(saddr, CHUNK, 1024);
+__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) {     // MN-major, SW128, 8 KB atoms
+  return smem_desc_sw128(saddr, VCH, 1024);
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+// Word q (0..3) of a node's visibility mask, without dynamic register indexing.
+__device__ __forceinline__ uint32_t mask_word(const uint32_t (&w)[4], int q) {
+  return q == 0 ? w[0] : (q == 1 ? w[1] : (q == 2 ? w[2] : w[3]));
+}
+
+__device__ __forceinline__ float max4(float a, float b, float c, float d) {
+  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
+// ====================================================================== QK CTA roles
+// TMA producer: Q chunks 7 and 8 once, then the K ring.
+__device__ __forceinline__ void qk_producer(const Ctx& cx, const CUtensorMap* tm_qa,
+                                            const CUtensorMap* tm_qr, const CUtensorMap* tm_c,
+                                            const CUtensorMap* tm_r, int qrow0, int64_t krow0,
+                                            int ntiles) {
+  const uint32_t base = cx.base;
+  mbar_arrive_expect_tx(cx.bar(Q_FULL), 2 * CHUNK);
+  tma_load_2d(base + Q_OFF, tm_qa, 7 * KC, qrow0, cx.bar(Q_FULL));
+  tma_load_2d(base + Q_OFF + CHUNK, tm_qr, 0, qrow0, cx.bar(Q_FULL));
+  uint32_t it = 0;
+  bool ok = true;
+  for (int t = 0; t < ntiles && ok; ++t) {
+    const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN);
+    for (int c = 0; c < NCHUNK; ++c, ++it) {
+      const uint32_t st = it % NK, k = it / NK;
+      if (!(ok = wait_bar(cx, cx.bar(K_EMPTY + st), (k & 1u) ^ 1u))) break;
+      mbar_arrive_expect_tx(cx.bar(K_FULL + st), CHUNK);
+      if (c < 8) tma_load_2d(base + K_OFF + st * CHUNK, tm_c, c * KC, krow, cx.bar(K_FULL + st));
+      else tma_load_2d(base + K_OFF + st * CHUNK, tm_r, 0, krow, cx.bar(K_FULL + st));
+    }
+  }
+  // every armed stage must have landed before the CTA may exit
+  wait_bar(cx, cx.bar(Q_FULL), 0);
+  for (uint32_t j = (it > NK ? it - NK : 0); j < it; ++j)
+    wait_bar(cx, cx.bar(K_FULL + j % NK), (j / NK) & 1u);
+}
+
+// MMA issuer: S[t % 2] = Q K^T (A from TMEM for chunks 0..6, from shared memory for 7, 8).
+__device__ __forceinline__ void qk_mma(const Ctx& cx, uint32_t tmem, int ntiles) {
+  const uint32_t base = cx.base;
+  bool ok = wait_bar(cx, cx.bar(Q_FULL), 0) && wait_bar(cx, cx.bar(QT_FULL), 0);
+  tc_fence_after();
+  uint32_t it = 0;
+  for (int t = 0; t < ntiles && ok; ++t) {
+    const uint32_t sb = t & 1;
+    if (!(ok = wait_bar(cx, cx.bar(S_EMPTY + sb), ((t >> 1) & 1) ^ 1))) break;
+    tc_fence_after();
+    const uint32_t d = tmem + TS + sb * BN;
+    for (int c = 0; c < NCHUNK; ++c, ++it) {
+      const uint32_t st = it % NK;
+      if (!(ok = wait_bar(cx, cx.bar(K_FULL + st), (it / NK) & 1u))) break;
+      tc_fence_after();
+      const uint32_t b0 = base + K_OFF + st * CHUNK;
+      if (c < NQT) {
+#pragma unroll
+        for (int kk = 0; kk < KC / 16; ++kk)
+          mma_bf16_ts(d, tmem + TQ + c * 32 + kk * 8, desc_k(b0 + kk * 32), IDESC_QK, (c | kk) != 0);
+      } else {
+        const uint32_t a0 = base + Q_OFF + (c - NQT) * CHUNK;
+#pragma unroll
+        for (int kk = 0; kk < KC / 16; ++kk)
+          mma_bf16_ss(d, desc_k(a0 + kk * 32), desc_k(b0 + kk * 32), IDESC_QK, 1u);
+      }
+      tc_commit(cx.bar(K_EMPTY + st));
+    }
+    if (ok) tc_commit(cx.bar(S_FULL + sb));
+  }
+  tc_commit(cx.bar(DRAIN));
+  wait_bar(cx, cx.bar(DRAIN), 0);
+}
+
+// Softmax groups: thread (g, r) owns row r and key columns [64 g, 64 g + 64) of every tile.
+__device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8_t* gbase,
+                                           uint32_t tmem, int b, int mt, int sp, int64_t L,
+                                           int64_t kbeg, int ntiles) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = (warp - 2) >> 2;
+  const int quad = warp & 3;
+  const int r = quad * 32 + lane;
+  const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+  const int n = p.n, H = p.H, rows_req = n * H;
+  const int R = mt * BM + r;
+  const bool valid = R < rows_req;
+  const int node = valid ? R / H : 0;
+  float* xch = reinterpret_cast<float*>(gbase + OFF_XCH);
+
+  // ---- Q chunks 0..6 of this row into TMEM (group 0: chunks 0..3, group 1: 4..6)
+  {
+    const int64_t grow = (int64_t)b * rows_req + R;
+    const bool in_range = R < rows_req;
+    const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + grow * KD_D_C);
+    const int c0 = g == 0 ? 0 : 4, c1 = g == 0 ? 4 : NQT;
+    for (int c = c0; c < c1; ++c) {
+      uint32_t v[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint4 x = in_range ? src[c * 8 + q] : make_uint4(0u, 0u, 0u, 0u);
+        v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+      }
+      tmem_st32(lane_addr + TQ + c * 32, v);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(cx.bar(QT_FULL));
+  }
+
+  const int W = p.W;
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) w[q] = q < W ? p.vis[((size_t)b * n + node) * W + q] : 0u;
+  if (g == 0 && valid && sp == 0 && (R % H) == 0) {
+    const int depth = __popc(w[0]) + __popc(w[1]) + __popc(w[2]) + __popc(w[3]) - 1;
+    if (!(w[0] & 1u) || !((mask_word(w, node >> 5) >> (node & 31)) & 1u)) raise_dev_error(p.err, KD_DEV_BAD_MASK);
+    if (p.positions && p.positions[(size_t)b * n + node] != (int32_t)(L + depth))
+      raise_dev_error(p.err, KD_DEV_BAD_POSITION);
+  }
+  const uint32_t peer_p = map_to_rank(cx.base + P_OFF, cx.peer);
+  const uint32_t peer_ctrl = map_to_rank(cx.base, cx.peer);
+  float m_ref = -INFINITY, l_part = 0.f;
+  bool ok = true;
+  for (int t = 0; t < ntiles && ok; ++t) {
+    const uint32_t sb = t & 1;
+    if (!(ok = wait_group(cx, cx.bar(S_FULL + sb), (t >> 1) & 1))) break;
+    tc_fence_after();
+    float x[64];
+    {
+      uint32_t u0[32], u1[32];
+      tmem_ld32(lane_addr + TS + sb * BN + g * 64, u0);
+      tmem_ld32(lane_addr + TS + sb * BN + g * 64 + 32, u1);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        x[k] = __uint_as_float(u0[k]) * p.scale_log2;
+        x[32 + k] = __uint_as_float(u1[k]) * p.scale_log2;
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(cx.bar(S_EMPTY + sb));
+    // mask: only keys at or beyond L need it
+    const int64_t kt = kbeg + (int64_t)t * BN + g * 64;
+    if (kt + 64 > L) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const int64_t k = kt + c - L;
+        bool vis_c = true;
+        if (k >= 0) vis_c = (k < n) && ((mask_word(w, (int)k >> 5) >> ((int)k & 31)) & 1u);
+        if (!vis_c) x[c] = -INFINITY;
+      }
+    }
+    float mx[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+    for (int c = 4; c < 64; c += 4) {
+      mx[0] = fmaxf(mx[0], x[c]); mx[1] = fmaxf(mx[1], x[c + 1]);
+      mx[2] = fmaxf(mx[2], x[c + 2]); mx[3] = fmaxf(mx[3], x[c + 3]);
+    }
+    xch[g * BM + r] = max4(mx[0], mx[1], mx[2], mx[3]);
+    named_bar_sync(1, GROUP);
+    const float tmax = fmaxf(xch[r], xch[BM + r]);
+    float alpha = 1.f;
+    bool rescale_row = false;
+    if (tmax > m_ref + RESCALE_THRESHOLD) {
+      if (m_ref != -INFINITY) {
+        alpha = ex2(m_ref - tmax);
+        rescale_row = true;
+      } else {
+        alpha = 0.f;
+      }
+      l_part *= alpha;
+      m_ref = tmax;
+    }
+    const float mb = m_ref == -INFINITY ? 0.f : m_ref;
+    float rs[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const float p0 = ex2(x[2 * c] - mb), p1 = ex2(x[2 * c + 1] - mb);
+      rs[c & 3] += p0 + p1;
+      pk[c] = pack_bf16x2(p0, p1);
+    }
+    l_part += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+    // P slot sb is free once the PV MMAs of tile t-2 completed
+    if (!(ok = wait_group(cx, cx.bar(P_FREE + sb), ((t >> 1) & 1) ^ 1))) break;
+    const uint32_t prow = peer_p + sb * PSLOT + g * (BM * 128) + (uint32_t)r * 128u;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      st_cluster_v4(prow + ((q ^ (r & 7)) << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    if (g == 0) st_cluster_u32(peer_ctrl + OFF_ALPHA + (sb * BM + r) * 4, __float_as_uint(alpha));
+    fence_proxy_async_cluster();
+    const bool any = named_bar_red_or(1, GROUP, rescale_row);
+    if (threadIdx.x == 64) {
+      st_cluster_u32(peer_ctrl + OFF_FLAG + sb * 4, any ? 1u : 0u);
+      mbar_arrive_remote(peer_ctrl + 8u * P_FULL + 8u * sb);
+    }
+  }
+  // final row statistics for the epilogue: l = both groups' partial sums
+  named_bar_sync(1, GROUP);
+  xch[g * BM + r] = l_part;
+  named_bar_sync(1, GROUP);
+  if (g == 0) {
+    st_cluster_u32(peer_ctrl + OFF_MFIN + r * 4, __float_as_uint(m_ref));
+    st_cluster_u32(peer_ctrl + OFF_LFIN + r * 4, __float_as_uint(xch[r] + xch[BM + r]));
+  }
+  named_bar_sync(1, GROUP);
+  if (threadIdx.x == 64) {
+    mbar_arrive_remote(peer_ctrl + 8u * STATS);
+    // the last P_FREE arrivals come from the peer's MMA completion: wait for them
+    if (ok)
+      for (int t = (ntiles > 2 ? ntiles - 2 : 0); t < ntiles; ++t)
+        wait_bar(cx, cx.bar(P_FREE + (t & 1)), (t >> 1) & 1);
+  }
+}
+
+// ====================================================================== PV CTA roles
+__device__ __forceinline__ void pv_producer(const Ctx& cx, const CUtensorMap* tm_v, int64_t krow0,
+                                            int ntiles) {
+  bool ok = true;
+  uint32_t gi = 0;
+  for (int t = 0; t < ntiles && ok; ++t) {
+    for (int kh = 0; kh < BN / VKEYS && ok; ++kh) {
+      const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN + kh * VKEYS);
+      for (int hh = 0; hh < 2; ++hh, ++gi) {
+        const uint32_t gs = gi % NVG, k = gi / NVG;
+        if (!(ok = wait_bar(cx, cx.bar(V_EMPTY + gs), (k & 1u) ^ 1u))) break;
+        mbar_arrive_expect_tx(cx.bar(V_FULL + gs), VG);
+        for (int q = 0; q < 4; ++q)
+          tma_load_2d(cx.base + V_OFF + gs * VG + q * VCH, tm_v, (hh * 4 + q) * KC, krow,
+                      cx.bar(V_FULL + gs));
+      }
+    }
+  }
+  for (uint32_t j = (gi > NVG ? gi - NVG : 0); j < gi; ++j)
+    wait_bar(cx, cx.bar(V_FULL + j % NVG), (j / NVG) & 1u);
+}
+
+__device__ __forceinline__ void pv_mma(const Ctx& cx, uint8_t* gbase, uint32_t tmem, int64_t kbeg,
+                                       int64_t nkeys, int ntiles) {
+  const int lane = threadIdx.x & 31;
+  volatile uint32_t* ctrl = reinterpret_cast<volatile uint32_t*>(gbase);
+  bool ok = true;
+  uint32_t gi = 0, nres = 0;
+  for (int t = 0; t < ntiles && ok; ++t) {
+    const uint32_t sb = t & 1;
+    if (!(ok = wait_warp(cx, cx.bar(P_FULL + sb), (t >> 1) & 1, true))) break;
+    fence_proxy_async_cta();
+    const uint32_t flag = ctrl[(OFF_FLAG >> 2) + sb];
+    if (flag && t > 0) {
+      // every earlier PV MMA must be done before O is rescaled
+      if (!(ok = wait_warp(cx, cx.bar(PV_TILE), (t - 1) & 1))) break;
+      if (lane == 0) {
+        ctrl[OFF_EVTYPE >> 2] = 1u;
+        ctrl[OFF_EVTILE >> 2] = sb;
+        mbar_arrive(cx.bar(EVENT));
+      }
+      if (!(ok = wait_warp(cx, cx.bar(CORR_DONE), nres & 1u))) break;
+      ++nres;
+    }
+    tc_fence_after();
+    const int64_t kt = kbeg + (int64_t)t * BN;
+    const int nvalid = (int)((nkeys - kt) < BN ? (nkeys - kt) : BN);
+    for (int kh = 0; kh < BN / VKEYS && ok; ++kh) {
+      const int nv = min(max(nvalid - kh * VKEYS, 0), VKEYS);
+      for (int hh = 0; hh < 2 && ok; ++hh, ++gi) {
+        const uint32_t gs = gi % NVG;
+        if (!(ok = wait_warp(cx, cx.bar(V_FULL + gs), (gi / NVG) & 1u))) break;
+        if (nv < VKEYS) {
+          // rows past the request's last key may hold anything (even NaN bit
+          // patterns); P is 0 there but 0 * NaN is not, so clear them
+          uint4* vg = reinterpret_cast<uint4*>(gbase + V_OFF + gs * VG);
+          const int per_chunk = (VKEYS - nv) * 8;
+          for (int idx = lane; idx < 4 * per_chunk; idx += 32) {
+            const int q = idx / per_chunk, e = idx % per_chunk;
+            vg[q * (VCH / 16) + nv * 8 + e] = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_cta();
+          __syncwarp();
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t pa = cx.base + P_OFF + sb * PSLOT + kh * (BM * 128);
+          const uint32_t vb = cx.base + V_OFF + gs * VG;
+#pragma unroll
+          for (int ks = 0; ks < VKEYS / 16; ++ks)
+            mma_bf16_ss(tmem + hh * 256, desc_k(pa + ks * 32), desc_mn(vb + ks * 2048), IDESC_PV,
+                        (t > 0 || kh > 0 || ks > 0) ? 1u : 0u);
+          tc_commit(cx.bar(V_EMPTY + gs));
+        }
+        __syncwarp();
+      }
+    }
+    if (ok && lane == 0) {
+      tc_commit(cx.bar(PV_TILE));
+      tc_commit_mc(cx.bar(P_FREE + sb), (uint16_t)(1u << cx.peer));
+    }
+    __syncwarp();
+  }
+  if (lane == 0) {
+    if (ntiles > 0) tc_commit(cx.bar(O_DONE));
+    else mbar_arrive(cx.bar(O_DONE));
+    ctrl[OFF_EVTYPE >> 2] = 2u;
+    mbar_arrive(cx.bar(EVENT));
+  }
+  __syncwarp();
+}
+
+// Correction / epilogue groups: thread (g, r) owns row r, O columns [256 g, 256 g + 256).
+__device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, uint8_t* gbase,
+                                            uint32_t tmem, int b, int mt, int sp, int ntiles) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = (warp - 2) >> 2;
+  const int quad = warp & 3;
+  const int r = quad * 32 + lane;
+  const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16) + g * 256;
+  volatile uint32_t* ctrl = reinterpret_cast<volatile uint32_t*>(gbase);
+  const volatile float* fctrl = reinterpret_cast<const volatile float*>(gbase);
+  bool ok = true;
+  uint32_t nev = 0;
+  while (true) {
+    if (!(ok = wait_group(cx, cx.bar(EVENT), nev & 1u))) break;
+    ++nev;
+    if (ctrl[OFF_EVTYPE >> 2] != 1u) break;
+    const uint32_t sb = ctrl[OFF_EVTILE >> 2];
+    const float a = fctrl[(OFF_ALPHA >> 2) + sb * BM + r];
+    tc_fence_after();
+    uint32_t v[32];
+    for (int c = 0; c < 256 / 32; ++c) {
+      tmem_ld32(lane_addr + c * 32, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * a);
+      tmem_st32(lane_addr + c * 32, v);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(cx.bar(CORR_DONE));
+  }
+  if (ok) ok = wait_group(cx, cx.bar(STATS), 0, true);
+  if (ok) ok = wait_group(cx, cx.bar(O_DONE), 0);
+  tc_fence_after();
+  const float m = ok ? fctrl[(OFF_MFIN >> 2) + r] : 0.f;
+  const float l = ok ? fctrl[(OFF_LFIN >> 2) + r] : 0.f;
+  const int rows_req = p.n * p.H;
+  const int R = mt * BM + r;
+  const bool valid = ok && R < rows_req;
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  const bool have_o = ntiles > 0;
+  const int64_t grow = (int64_t)b * rows_req + R;
+  const int64_t prow = ((int64_t)sp * p.B * rows_req) + grow;
+  uint32_t v0[32], v1[32];
+  for (int c = 0; c < 256 / 64; ++c) {
+    if (have_o && ok) {
+      tmem_ld32(lane_addr + c * 64, v0);
+      tmem_ld32(lane_addr + c * 64 + 32, v1);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int k = 0; k < 32; ++k) v0[k] = v1[k] = 0u;
+    }
+    if (!valid) continue;
+    const int col = g * 256 + c * 64;
+    if (p.splits == 1) {
+      uint4* dst = reinterpret_cast<uint4*>(p.out + grow * KD_D_C + col);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t* v = q < 4 ? v0 : v1;
+        const int o = (q & 3) * 8;
+        dst[q] = make_uint4(pack_bf16x2(__uint_as_float(v[o + 0]) * inv, __uint_as_float(v[o + 1]) * inv),
+                            pack_bf16x2(__uint_as_float(v[o + 2]) * inv, __uint_as_float(v[o + 3]) * inv),
+                            pack_bf16x2(__uint_as_float(v[o + 4]) * inv, __uint_as_float(v[o + 5]) * inv),
+                            pack_bf16x2(__uint_as_float(v[o + 6]) * inv, __uint_as_float(v[o + 7]) * inv));
+      }
+    } else {
+      float4* dst = reinterpret_cast<float4*>(p.part_o + prow * KD_D_C + col);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const uint32_t* v = q < 8 ? v0 : v1;
+        const int o = (q & 7) * 4;
+        dst[q] = make_float4(__uint_as_float(v[o]) * inv, __uint_as_float(v[o + 1]) * inv,
+                             __uint_as_float(v[o + 2]) * inv, __uint_as_float(v[o + 3]) * inv);
+      }
+    }
+  }
+  if (valid && g == 0) {
+    const float lse_v = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    if (p.splits == 1) p.lse[grow] = lse_v;
+    else p.part_lse[prow] = lse_v;
+  }
+  tc_fence_before();
+}
+
+// ====================================================================== kernel
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant__ CUtensorMap tm_qr,
                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
-               const __grid_constant__ Params p) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -197,8 +602,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   const int ntiles = t1 - t0;
   const int64_t kbeg = (int64_t)t0 * BN;                    // request-relative first key
   const int64_t krow0 = (int64_t)b * p.cap + kbeg;          // cache row of the first key
-  const int rows_req = n * H;
-  const int qrow0 = b * rows_req + mt * BM;
+  const int qrow0 = b * n * H + mt * BM;
 
   Ctx cx;
   cx.base = base;
@@ -207,30 +611,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   cx.err = p.err;
 
   if (threadIdx.x == 0) {
-    const uint32_t counts[NBAR] = {
-        1,                   // Q_FULL
-        1, 1, 1, 1,          // K_FULL
-        1, 1, 1, 1,          // K_EMPTY
-        1, 1,                // S_FULL
-        128, 128,            // S_EMPTY
-        1, 1,                // P_FREE
-        1, 1,                // V_FULL
-        1, 1,                // V_EMPTY
-        1, 1,                // P_FULL
-        1,                   // PV_TILE
-        1,                   // O_DONE
-        1,                   // EVENT
-        128,                 // CORR_DONE
-        1,                   // STATS
-        1};                  // DRAIN
-    static_assert(sizeof(counts) / sizeof(counts[0]) == NBAR, "barrier counts");
-    for (int i = 0; i < NBAR; ++i) mbar_init(cx.bar(i), counts[i]);
+    for (int i = 0; i < NBAR; ++i) {
+      uint32_t cnt = 1;
+      if (i == QT_FULL || i == S_EMPTY || i == S_EMPTY + 1 || i == CORR_DONE) cnt = GROUP;
+      mbar_init(cx.bar(i), cnt);
+    }
     *cx.abort_flag = 0u;
     fence_mbar_init();
   }
-  const uint32_t tmem_cols = rank == 0 ? 256u : 512u;
   if (warp == 1) {
-    tmem_alloc(base + OFF_TMEM, tmem_cols);
+    tmem_alloc(base + OFF_TMEM, 512);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -238,6 +628,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
     tma_prefetch_desc(&tm_qr);
     tma_prefetch_desc(&tm_c);
     tma_prefetch_desc(&tm_r);
+    tma_prefetch_desc(&tm_v);
   }
   tc_fence_before();
   cluster_sync();
@@ -245,317 +636,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + OFF_TMEM);
 
   if (rank == 0) {
-    // ======================================================= QK CTA
     if (warp == 0) {
-      // ---------------- TMA producer: Q once, then K chunks
-      if (lane == 0 && ntiles > 0) {
-        bool ok = true;
-        mbar_arrive_expect_tx(cx.bar(Q_FULL), NCHUNK * CHUNK);
-        for (int c = 0; c < 8; ++c)
-          tma_load_2d(base + Q_OFF + c * CHUNK, &tm_qa, c * KC, qrow0, cx.bar(Q_FULL));
-        tma_load_2d(base + Q_OFF + 8 * CHUNK, &tm_qr, 0, qrow0, cx.bar(Q_FULL));
-        uint32_t it = 0;
-        for (int t = 0; t < ntiles && ok; ++t) {
-          const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN);
-          for (int c = 0; c < NCHUNK; ++c, ++it) {
-            const uint32_t st = it % NK, k = it / NK;
-            if (!(ok = wait_bar(cx, cx.bar(K_EMPTY + st), (k & 1u) ^ 1u))) break;
-            mbar_arrive_expect_tx(cx.bar(K_FULL + st), CHUNK);
-            if (c < 8) tma_load_2d(base + K_OFF + st * CHUNK, &tm_c, c * KC, krow, cx.bar(K_FULL + st));
-            else tma_load_2d(base + K_OFF + st * CHUNK, &tm_r, 0, krow, cx.bar(K_FULL + st));
-          }
-        }
-        // drain: every armed stage must have landed before the CTA can exit
-        wait_bar(cx, cx.bar(Q_FULL), 0);
-        for (uint32_t j = (it > NK ? it - NK : 0); j < it; ++j)
-          wait_bar(cx, cx.bar(K_FULL + j % NK), (j / NK) & 1u);
-      }
+      if (lane == 0 && ntiles > 0) qk_producer(cx, &tm_qa, &tm_qr, &tm_c, &tm_r, qrow0, krow0, ntiles);
     } else if (warp == 1) {
-      // ---------------- MMA issuer: S[sb] = Q K^T
-      if (lane == 0 && ntiles > 0) {
-        bool ok = wait_bar(cx, cx.bar(Q_FULL), 0);
-        tc_fence_after();
-        uint32_t it = 0;
-        for (int t = 0; t < ntiles && ok; ++t) {
-          const uint32_t sb = t & 1;
-          if (!(ok = wait_bar(cx, cx.bar(S_EMPTY + sb), ((t >> 1) & 1) ^ 1))) break;
-          tc_fence_after();
-          const uint32_t d = tmem + sb * BN;
-          for (int c = 0; c < NCHUNK; ++c, ++it) {
-            const uint32_t st = it % NK;
-            if (!(ok = wait_bar(cx, cx.bar(K_FULL + st), (it / NK) & 1u))) break;
-            tc_fence_after();
-            const uint32_t a0 = base + Q_OFF + c * CHUNK, b0 = base + K_OFF + st * CHUNK;
-#pragma unroll
-            for (int kk = 0; kk < KC / 16; ++kk)
-              mma_bf16_ss(d, desc_k(a0 + kk * 32), desc_k(b0 + kk * 32), IDESC_QK, (c | kk) != 0);
-            tc_commit(cx.bar(K_EMPTY + st));
-          }
-          if (ok) tc_commit(cx.bar(S_FULL + sb));
-        }
-        tc_commit(cx.bar(DRAIN));
-        wait_bar(cx, cx.bar(DRAIN), 0);
-      }
+      if (lane == 0 && ntiles > 0) qk_mma(cx, tmem, ntiles);
       __syncwarp();
     } else {
-      // ---------------- softmax group (warps 2..5): one thread per query row
-      const int quad = warp & 3;
-      const int r = quad * 32 + lane;
-      const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-      const int R = mt * BM + r;
-      const bool valid = R < rows_req;
-      const int node = valid ? R / H : 0;
-      const int W = p.W;
-      uint32_t w[4] = {0u, 0u, 0u, 0u};
-      for (int q = 0; q < W; ++q) w[q] = p.vis[((size_t)b * n + node) * W + q];
-      if (valid && sp == 0 && (R % H) == 0) {
-        int depth = -1;
-        for (int q = 0; q < W; ++q) depth += __popc(w[q]);
-        if (!(w[0] & 1u) || !((w[node >> 5] >> (node & 31)) & 1u)) raise_dev_error(p.err, KD_DEV_BAD_MASK);
-        if (p.positions && p.positions[(size_t)b * n + node] != (int32_t)(L + depth))
-          raise_dev_error(p.err, KD_DEV_BAD_POSITION);
-      }
-      const uint32_t peer_p = map_to_rank(base + P_OFF, cx.peer);
-      const uint32_t peer_ctrl = map_to_rank(base, cx.peer);
-      float m_ref = -INFINITY, l = 0.f;
-      bool ok = true;
-      for (int t = 0; t < ntiles && ok; ++t) {
-        const uint32_t sb = t & 1;
-        if (!(ok = wait_group(cx, cx.bar(S_FULL + sb), (t >> 1) & 1, 1))) break;
-        tc_fence_after();
-        float x[BN];
-        {
-          uint32_t v[32];
-#pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            tmem_ld32(lane_addr + sb * BN + c * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) x[c * 32 + k] = __uint_as_float(v[k]) * p.scale_log2;
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(cx.bar(S_EMPTY + sb));
-        // mask: only keys at or beyond L need it
-        const int64_t kt = kbeg + (int64_t)t * BN;
-        if (kt + BN > L) {
-#pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const int64_t k = kt + c - L;
-            bool vis_c = true;
-            if (k >= 0) vis_c = (k < n) && ((w[(int)k >> 5] >> ((int)k & 31)) & 1u);
-            if (!vis_c) x[c] = -INFINITY;
-          }
-        }
-        float tmax = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < BN; ++c) tmax = fmaxf(tmax, x[c]);
-        float alpha = 1.f;
-        bool rescale_row = false;
-        if (tmax > m_ref + RESCALE_THRESHOLD) {
-          if (m_ref != -INFINITY) {
-            alpha = ex2(m_ref - tmax);
-            rescale_row = true;
-          } else {
-            alpha = 0.f;
-          }
-          l *= alpha;
-          m_ref = tmax;
-        }
-        const float mb = m_ref == -INFINITY ? 0.f : m_ref;
-        float rs = 0.f;
-        uint32_t pk[BN / 2];
-#pragma unroll
-        for (int c = 0; c < BN / 2; ++c) {
-          const float p0 = ex2(x[2 * c] - mb), p1 = ex2(x[2 * c + 1] - mb);
-          rs += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
-        }
-        l += rs;
-        // P slot sb is free once the PV MMAs of tile t-2 completed
-        if (!(ok = wait_group(cx, cx.bar(P_FREE + sb), ((t >> 1) & 1) ^ 1, 1))) break;
-        const uint32_t prow = peer_p + sb * PSLOT + (uint32_t)r * 128u;
-#pragma unroll
-        for (int q = 0; q < BN / 8; ++q) {
-          const uint32_t atom = q >> 3, chunk = (q & 7) ^ (r & 7);
-          st_cluster_v4(prow + atom * (BM * 128) + chunk * 16, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
-                        pk[4 * q + 3]);
-        }
-        st_cluster_u32(peer_ctrl + OFF_ALPHA + (sb * BM + r) * 4, __float_as_uint(alpha));
-        fence_proxy_async_cluster();
-        const bool any = named_bar_red_or(1, 128, rescale_row);
-        if (r == 0) {
-          st_cluster_u32(peer_ctrl + OFF_FLAG + sb * 4, any ? 1u : 0u);
-          mbar_arrive_remote(peer_ctrl + 8u * P_FULL + 8u * sb);
-        }
-      }
-      // final row statistics for the epilogue
-      st_cluster_u32(peer_ctrl + OFF_MFIN + r * 4, __float_as_uint(m_ref));
-      st_cluster_u32(peer_ctrl + OFF_LFIN + r * 4, __float_as_uint(l));
-      named_bar_sync(1, 128);
-      if (r == 0) mbar_arrive_remote(peer_ctrl + 8u * STATS);
-      // the last P_FREE arrivals come from the peer's MMA completion: wait for them
-      if (ok && r == 0)
-        for (int t = (ntiles > 2 ? ntiles - 2 : 0); t < ntiles; ++t)
-          wait_bar(cx, cx.bar(P_FREE + (t & 1)), (t >> 1) & 1);
+      qk_softmax(cx, p, gbase, tmem, b, mt, sp, L, kbeg, ntiles);
     }
   } else {
-    // ======================================================= PV CTA
     if (warp == 0) {
-      // ---------------- TMA producer: V groups (128 keys x 256 latent columns)
-      if (lane == 0) {
-        bool ok = true;
-        uint32_t gi = 0;
-        for (int t = 0; t < ntiles && ok; ++t) {
-          const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN);
-          for (int hh = 0; hh < 2; ++hh, ++gi) {
-            const uint32_t g = gi % NVG, k = gi / NVG;
-            if (!(ok = wait_bar(cx, cx.bar(V_EMPTY + g), (k & 1u) ^ 1u))) break;
-            mbar_arrive_expect_tx(cx.bar(V_FULL + g), VG);
-            for (int q = 0; q < 4; ++q)
-              tma_load_2d(base + V_OFF + g * VG + q * CHUNK, &tm_c, (hh * 4 + q) * KC, krow,
-                          cx.bar(V_FULL + g));
-          }
-        }
-        for (uint32_t j = (gi > NVG ? gi - NVG : 0); j < gi; ++j)
-          wait_bar(cx, cx.bar(V_FULL + j % NVG), (j / NVG) & 1u);
-      }
+      if (lane == 0) pv_producer(cx, &tm_v, krow0, ntiles);
     } else if (warp == 1) {
-      // ---------------- MMA issuer: O += P V
-      volatile uint32_t* ctrl = reinterpret_cast<volatile uint32_t*>(gbase);
-      bool ok = true;
-      uint32_t gi = 0, nres = 0;
-      for (int t = 0; t < ntiles && ok; ++t) {
-        const uint32_t sb = t & 1;
-        if (!(ok = wait_warp(cx, cx.bar(P_FULL + sb), (t >> 1) & 1, true))) break;
-        fence_proxy_async_cta();
-        const uint32_t flag = ctrl[(OFF_FLAG >> 2) + sb];
-        if (flag && t > 0) {
-          // every earlier PV MMA must be done before O is rescaled
-          if (!(ok = wait_warp(cx, cx.bar(PV_TILE), (t - 1) & 1))) break;
-          if (lane == 0) {
-            ctrl[OFF_EVTYPE >> 2] = 1u;
-            ctrl[OFF_EVTILE >> 2] = sb;
-            mbar_arrive(cx.bar(EVENT));
-          }
-          if (!(ok = wait_warp(cx, cx.bar(CORR_DONE), nres & 1u))) break;
-          ++nres;
-        }
-        tc_fence_after();
-        const int64_t kt = kbeg + (int64_t)t * BN;
-        const int nvalid = (int)((nkeys - kt) < BN ? (nkeys - kt) : BN);
-        for (int hh = 0; hh < 2 && ok; ++hh, ++gi) {
-          const uint32_t g = gi % NVG;
-          if (!(ok = wait_warp(cx, cx.bar(V_FULL + g), (gi / NVG) & 1u))) break;
-          if (nvalid < BN) {
-            // rows past the request's last key may hold anything (even NaN bit
-            // patterns); P is 0 there but 0 * NaN is not, so clear them
-            uint4* vg = reinterpret_cast<uint4*>(gbase + V_OFF + g * VG);
-            const int per_chunk = (BN - nvalid) * 8;
-            for (int idx = lane; idx < 4 * per_chunk; idx += 32) {
-              const int q = idx / per_chunk, e = idx % per_chunk;
-              vg[q * (CHUNK / 16) + nvalid * 8 + e] = make_uint4(0u, 0u, 0u, 0u);
-            }
-            fence_proxy_async_cta();
-            __syncwarp();
-          }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t pa = base + P_OFF + sb * PSLOT, vb = base + V_OFF + g * VG;
-#pragma unroll
-            for (int ks = 0; ks < BN / 16; ++ks)
-              mma_bf16_ss(tmem + hh * 256, desc_k(pa + (ks >> 2) * (BM * 128) + (ks & 3) * 32),
-                          desc_mn(vb + ks * 2048), IDESC_PV, (t > 0 || ks > 0) ? 1u : 0u);
-            tc_commit(cx.bar(V_EMPTY + g));
-          }
-          __syncwarp();
-        }
-        if (ok && lane == 0) {
-          tc_commit(cx.bar(PV_TILE));
-          tc_commit_mc(cx.bar(P_FREE + sb), (uint16_t)(1u << cx.peer));
-        }
-        __syncwarp();
-      }
-      if (lane == 0) {
-        if (ntiles > 0) tc_commit(cx.bar(O_DONE));
-        else mbar_arrive(cx.bar(O_DONE));
-        ctrl[OFF_EVTYPE >> 2] = 2u;
-        mbar_arrive(cx.bar(EVENT));
-      }
-      __syncwarp();
+      pv_mma(cx, gbase, tmem, kbeg, nkeys, ntiles);
     } else {
-      // ---------------- correction / epilogue group (warps 2..5)
-      volatile uint32_t* ctrl = reinterpret_cast<volatile uint32_t*>(gbase);
-      const volatile float* fctrl = reinterpret_cast<const volatile float*>(gbase);
-      const int quad = warp & 3;
-      const int r = quad * 32 + lane;
-      const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-      bool ok = true;
-      uint32_t nev = 0;
-      while (true) {
-        if (!(ok = wait_group(cx, cx.bar(EVENT), nev & 1u, 1))) break;
-        ++nev;
-        if (ctrl[OFF_EVTYPE >> 2] != 1u) break;
-        const uint32_t sb = ctrl[OFF_EVTILE >> 2];
-        const float a = fctrl[(OFF_ALPHA >> 2) + sb * BM + r];
-        tc_fence_after();
-        uint32_t v[32];
-        for (int c = 0; c < 512 / 32; ++c) {
-          tmem_ld32(lane_addr + c * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * a);
-          tmem_st32(lane_addr + c * 32, v);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(cx.bar(CORR_DONE));
-      }
-      if (ok) ok = wait_group(cx, cx.bar(STATS), 0, 1, true);
-      if (ok) ok = wait_group(cx, cx.bar(O_DONE), 0, 1);
-      tc_fence_after();
-      const float m = ok ? fctrl[(OFF_MFIN >> 2) + r] : 0.f;
-      const float l = ok ? fctrl[(OFF_LFIN >> 2) + r] : 0.f;
-      const int R = mt * BM + r;
-      const bool valid = ok && R < rows_req;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const bool have_o = ntiles > 0;
-      const int64_t grow = (int64_t)b * rows_req + R;
-      const int64_t prow = ((int64_t)sp * p.B * rows_req) + grow;
-      uint32_t v[32];
-      for (int c = 0; c < 512 / 32; ++c) {
-        if (have_o && ok) {
-          tmem_ld32(lane_addr + c * 32, v);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = 0u;
-        }
-        if (!valid) continue;
-        if (p.splits == 1) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + grow * KD_D_C + c * 32);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t a0 = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
-            uint32_t a1 = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
-            uint32_t a2 = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
-            uint32_t a3 = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
-            dst[q] = make_uint4(a0, a1, a2, a3);
-          }
-        } else {
-          float4* dst = reinterpret_cast<float4*>(p.part_o + prow * KD_D_C + c * 32);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(v[4 * q]) * inv, __uint_as_float(v[4 * q + 1]) * inv,
-                                 __uint_as_float(v[4 * q + 2]) * inv, __uint_as_float(v[4 * q + 3]) * inv);
-        }
-      }
-      if (valid) {
-        const float lse_v = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-        if (p.splits == 1) p.lse[grow] = lse_v;
-        else p.part_lse[prow] = lse_v;
-      }
-      tc_fence_before();
+      pv_epilogue(cx, p, gbase, tmem, b, mt, sp, ntiles);
     }
   }
 
@@ -564,7 +659,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, tmem_cols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -581,13 +676,14 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 view [rows][inner] with `row_bytes` pitch, 64 x 128 boxes, 128-byte swizzle.
-static int make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint64_t row_bytes) {
+// 2-D bf16 view [rows][inner] with `row_bytes` pitch, 64 x box_rows boxes, 128-byte swizzle.
+static int make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+                    uint32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return KD_ELAUNCH;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {KC, 128};
+  cuuint32_t box[2] = {KC, box_rows};
   cuuint32_t es[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -608,7 +704,7 @@ static int active_pairs(int sms) {
   int pairs = sms / 2;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(NTHREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cudaLaunchAttribute at;
   at.id = cudaLaunchAttributeClusterDimension;
@@ -697,16 +793,18 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   }
   if (workspace_bytes_for(B, n, H, splits) > ws_bytes) return KD_ERANGE;
 
-  CUtensorMap tq, tr, tcv, tkr;
-  if ((st = tc::make_map(&tq, q_abs, KD_D_C, (uint64_t)rows, KD_D_C * 2))) return st;
-  if ((st = tc::make_map(&tr, q_rope, KD_D_R, (uint64_t)rows, KD_D_R * 2))) return st;
-  if ((st = tc::make_map(&tcv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2))) return st;
-  if ((st = tc::make_map(&tkr, k_rope, KD_D_R, (uint64_t)(B * cap), (uint64_t)sr * 2))) return st;
+  CUtensorMap tq, tr, tcv, tkr, tv;
+  if ((st = tc::make_map(&tq, q_abs, KD_D_C, (uint64_t)rows, KD_D_C * 2, tc::BM))) return st;
+  if ((st = tc::make_map(&tr, q_rope, KD_D_R, (uint64_t)rows, KD_D_R * 2, tc::BM))) return st;
+  if ((st = tc::make_map(&tcv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::BN))) return st;
+  if ((st = tc::make_map(&tkr, k_rope, KD_D_R, (uint64_t)(B * cap), (uint64_t)sr * 2, tc::BN))) return st;
+  if ((st = tc::make_map(&tv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::VKEYS))) return st;
 
   tc::Params prm;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   prm.cache_lens = cache_lens;
   prm.vis = vis;
+  prm.q_abs = q_abs;
   prm.positions = positions;
   prm.out = out;
   prm.lse = lse;
@@ -724,7 +822,8 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   prm.scale_log2 = scale * 1.4426950408889634f;
   const int64_t units = (int64_t)B * prm.mtiles * splits;
   if (2 * units > INT32_MAX) return KD_EINVAL;
-  tc::attn_tc_kernel<<<dim3((unsigned)(2 * units)), 192, tc::SMEM_BYTES, stream>>>(tq, tr, tcv, tkr, prm);
+  tc::attn_tc_kernel<<<dim3((unsigned)(2 * units)), tc::NTHREADS, tc::SMEM_BYTES, stream>>>(tq, tr, tcv, tkr, tv,
+                                                                                         prm);
   st = launch_status("attn_tc_kernel");
   if (st || splits == 1) return st;
   return launch_combine(prm.part_o, prm.part_lse, cache_lens, B, n, H, cap, splits, out, lse, stream);
