@@ -142,7 +142,7 @@ struct Ctx {
   __device__ uint32_t bar(int i) const { return base + 8u * (uint32_t)i; }
 };
 
-__device__ __noinline__ void abort_pair(const Ctx& cx) {
+__device__ __noinline__ void abort_pair(Ctx cx) {
   *cx.abort_flag = 1u;
   st_cluster_u32(map_to_rank(cx.base + OFF_ABORT, cx.peer), 1u);
   raise_dev_error(cx.err, KD_DEV_TIMEOUT);
@@ -546,22 +546,26 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, uint
     if (p.splits == 1) {
       uint4* dst = reinterpret_cast<uint4*>(p.out + grow * KD_D_C + col);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint32_t* v = q < 4 ? v0 : v1;
-        const int o = (q & 3) * 8;
-        dst[q] = make_uint4(pack_bf16x2(__uint_as_float(v[o + 0]) * inv, __uint_as_float(v[o + 1]) * inv),
-                            pack_bf16x2(__uint_as_float(v[o + 2]) * inv, __uint_as_float(v[o + 3]) * inv),
-                            pack_bf16x2(__uint_as_float(v[o + 4]) * inv, __uint_as_float(v[o + 5]) * inv),
-                            pack_bf16x2(__uint_as_float(v[o + 6]) * inv, __uint_as_float(v[o + 7]) * inv));
+      for (int q = 0; q < 4; ++q) {
+        const int o = q * 8;
+        dst[q] = make_uint4(pack_bf16x2(__uint_as_float(v0[o + 0]) * inv, __uint_as_float(v0[o + 1]) * inv),
+                            pack_bf16x2(__uint_as_float(v0[o + 2]) * inv, __uint_as_float(v0[o + 3]) * inv),
+                            pack_bf16x2(__uint_as_float(v0[o + 4]) * inv, __uint_as_float(v0[o + 5]) * inv),
+                            pack_bf16x2(__uint_as_float(v0[o + 6]) * inv, __uint_as_float(v0[o + 7]) * inv));
+        dst[4 + q] = make_uint4(pack_bf16x2(__uint_as_float(v1[o + 0]) * inv, __uint_as_float(v1[o + 1]) * inv),
+                                pack_bf16x2(__uint_as_float(v1[o + 2]) * inv, __uint_as_float(v1[o + 3]) * inv),
+                                pack_bf16x2(__uint_as_float(v1[o + 4]) * inv, __uint_as_float(v1[o + 5]) * inv),
+                                pack_bf16x2(__uint_as_float(v1[o + 6]) * inv, __uint_as_float(v1[o + 7]) * inv));
       }
     } else {
       float4* dst = reinterpret_cast<float4*>(p.part_o + prow * KD_D_C + col);
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const uint32_t* v = q < 8 ? v0 : v1;
-        const int o = (q & 7) * 4;
-        dst[q] = make_float4(__uint_as_float(v[o]) * inv, __uint_as_float(v[o + 1]) * inv,
-                             __uint_as_float(v[o + 2]) * inv, __uint_as_float(v[o + 3]) * inv);
+      for (int q = 0; q < 8; ++q) {
+        const int o = q * 4;
+        dst[q] = make_float4(__uint_as_float(v0[o]) * inv, __uint_as_float(v0[o + 1]) * inv,
+                             __uint_as_float(v0[o + 2]) * inv, __uint_as_float(v0[o + 3]) * inv);
+        dst[8 + q] = make_float4(__uint_as_float(v1[o]) * inv, __uint_as_float(v1[o + 1]) * inv,
+                                 __uint_as_float(v1[o + 2]) * inv, __uint_as_float(v1[o + 3]) * inv);
       }
     }
   }
