@@ -17,14 +17,14 @@
 // columns of an SM, leaving none for scores, so each unit of work runs on a
 // 2-CTA cluster with split roles:
 //   rank 0 ("QK" CTA): S = Q K^T into a double-buffered 2 x 128-column TMEM
-//       accumulator.  Seven of Q's nine 64-wide chunks sit in TMEM and feed the MMA
-//       as its A operand from tensor memory; the other two sit in shared memory.
-//       That leaves shared memory for an 11-stage ring of 128-key x 64-column K
-//       chunks (TMA, 128-byte swizzle), enough lead time to hide L2/HBM latency.
-//       Two 4-warp softmax groups split each S tile's columns, keep an online max
-//       with a lazy rescale threshold, and store bf16 P straight into rank 1's
-//       shared memory (st.shared::cluster) in the K-major swizzled layout the MMA
-//       reads.
+//       accumulator.  The eight 64-wide latent chunks of Q sit in the other 256
+//       TMEM columns and feed the MMA as its A operand from tensor memory; the rope
+//       chunk sits in shared memory.  That leaves shared memory for an 8-stage ring
+//       of 128-key x 64-column K chunks (TMA, 128-byte swizzle) and two P staging
+//       slots.  Two 4-warp softmax groups split each S tile's columns, keep an
+//       online max with a lazy rescale threshold, write bf16 P into a local staging
+//       slot in the K-major swizzled layout the MMA reads, and one thread moves the
+//       slot to rank 1 with a single bulk copy that completes on rank 1's barrier.
 //   rank 1 ("PV" CTA): O (128 x 512 fp32) in TMEM; V as 64-key x 256-column
 //       groups (four 64-column MN-major boxes) in a 4-deep ring; O += P V as
 //       M=128, N=256, K=16 MMAs; two 4-warp groups apply the rare O rescale and
@@ -61,17 +61,21 @@ constexpr int BN = 128;                 // keys per tile
 constexpr int KC = 64;                  // columns per 128-byte swizzle atom
 constexpr int NCHUNK = 9;               // 8 latent chunks + 1 rope chunk
 constexpr int CHUNK = BN * KC * 2;      // 16 KB: 128 rows x 64 bf16
-constexpr int NQT = 7;                  // Q chunks held in TMEM (the rest in shared memory)
-constexpr int NK = 11;                  // K ring stages
+constexpr int NQT = 8;                  // Q chunks held in TMEM (the rope chunk in shared memory)
+constexpr int NK = 8;                   // K ring stages
 constexpr int VKEYS = 64;               // keys per V group
 constexpr int VCH = VKEYS * KC * 2;     // 8 KB: 64 keys x 64 latent columns
 constexpr int VG = 4 * VCH;             // one V group: 64 keys x 256 latent columns
 constexpr int NVG = 4;                  // V ring depth
-constexpr int PSLOT = BM * BN * 2;      // one bf16 P tile (two 16 KB swizzle columns)
+constexpr int PBYTES = BM * BN * 2;     // one bf16 P tile (two 16 KB swizzle columns)
+constexpr int SLOT_ALPHA = PBYTES;      // f32 [128] per-row rescale factor
+constexpr int SLOT_FLAG = PBYTES + 512; // u32 rescale-needed flag
+constexpr int SLOT_COPY = PBYTES + 528; // bytes moved to the PV CTA per tile
+constexpr int PSLOT = PBYTES + 1024;    // slot stride (keeps 1024-byte alignment)
 
 // TMEM columns of the QK CTA
 constexpr uint32_t TS = 0;              // S[2]: 2 x 128 columns
-constexpr uint32_t TQ = 256;            // Q chunks 0..6: 7 x 32 columns
+constexpr uint32_t TQ = 256;            // Q chunks 0..7: 8 x 32 columns
 
 // control block (same offsets in both CTAs so the peer can address it)
 constexpr int CTRL = 4096;
@@ -98,15 +102,14 @@ constexpr int OFF_TMEM = 512;           // u32 TMEM base
 constexpr int OFF_ABORT = 516;          // u32 abort flag
 constexpr int OFF_EVTYPE = 520;         // u32 event type (1 rescale, 2 done)     [PV]
 constexpr int OFF_EVTILE = 524;         // u32 P slot of a rescale event           [PV]
-constexpr int OFF_FLAG = 528;           // u32 [2] rescale-needed flag per P slot  [PV, remote]
-constexpr int OFF_ALPHA = 1024;         // f32 [2][128] per-row rescale factor     [PV, remote]
 constexpr int OFF_MFIN = 2048;          // f32 [128] final running max (log2)      [PV, remote]
 constexpr int OFF_LFIN = 2560;          // f32 [128] final running sum             [PV, remote]
 constexpr int OFF_XCH = 3072;           // f32 [2][128] max / sum exchange         [QK, local]
 static_assert(NBAR * 8 <= OFF_TMEM, "barrier block overflow");
 
-constexpr int Q_OFF = CTRL;                           // Q chunks 7, 8
-constexpr int K_OFF = Q_OFF + (NCHUNK - NQT) * CHUNK;
+constexpr int Q_OFF = CTRL;                           // Q chunk 8 (rope)
+constexpr int STG_OFF = Q_OFF + (NCHUNK - NQT) * CHUNK; // P staging, 2 slots
+constexpr int K_OFF = STG_OFF + 2 * PSLOT;
 constexpr int QK_END = K_OFF + NK * CHUNK;
 constexpr int P_OFF = CTRL;
 constexpr int V_OFF = P_OFF + 2 * PSLOT;
@@ -200,9 +203,8 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const CUtensorMap* tm
                                             const CUtensorMap* tm_r, int qrow0, int64_t krow0,
                                             int ntiles) {
   const uint32_t base = cx.base;
-  mbar_arrive_expect_tx(cx.bar(Q_FULL), 2 * CHUNK);
-  tma_load_2d(base + Q_OFF, tm_qa, 7 * KC, qrow0, cx.bar(Q_FULL));
-  tma_load_2d(base + Q_OFF + CHUNK, tm_qr, 0, qrow0, cx.bar(Q_FULL));
+  mbar_arrive_expect_tx(cx.bar(Q_FULL), (NCHUNK - NQT) * CHUNK);
+  tma_load_2d(base + Q_OFF, tm_qr, 0, qrow0, cx.bar(Q_FULL));
   uint32_t it = 0;
   bool ok = true;
   for (int t = 0; t < ntiles && ok; ++t) {
@@ -221,7 +223,7 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const CUtensorMap* tm
     wait_bar(cx, cx.bar(K_FULL + j % NK), (j / NK) & 1u);
 }
 
-// MMA issuer: S[t % 2] = Q K^T (A from TMEM for chunks 0..6, from shared memory for 7, 8).
+// MMA issuer: S[t % 2] = Q K^T (A from TMEM for chunks 0..7, from shared memory for 8).
 __device__ __forceinline__ void qk_mma(const Ctx& cx, uint32_t tmem, int ntiles) {
   const uint32_t base = cx.base;
   bool ok = wait_bar(cx, cx.bar(Q_FULL), 0) && wait_bar(cx, cx.bar(QT_FULL), 0);
@@ -270,12 +272,12 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
   const int node = valid ? R / H : 0;
   float* xch = reinterpret_cast<float*>(gbase + OFF_XCH);
 
-  // ---- Q chunks 0..6 of this row into TMEM (group 0: chunks 0..3, group 1: 4..6)
+  // ---- Q chunks 0..7 of this row into TMEM (group 0: chunks 0..3, group 1: 4..7)
   {
     const int64_t grow = (int64_t)b * rows_req + R;
     const bool in_range = R < rows_req;
     const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + grow * KD_D_C);
-    const int c0 = g == 0 ? 0 : 4, c1 = g == 0 ? 4 : NQT;
+    const int c0 = g * 4, c1 = g * 4 + 4;
     for (int c = c0; c < c1; ++c) {
       uint32_t v[32];
 #pragma unroll
@@ -364,18 +366,21 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
       pk[c] = pack_bf16x2(p0, p1);
     }
     l_part += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-    // P slot sb is free once the PV MMAs of tile t-2 completed
+    // staging slot sb (and the peer's P slot sb) is free once the PV MMAs of tile t-2 completed
     if (!(ok = wait_group(cx, cx.bar(P_FREE + sb), ((t >> 1) & 1) ^ 1))) break;
-    const uint32_t prow = peer_p + sb * PSLOT + g * (BM * 128) + (uint32_t)r * 128u;
+    const uint32_t stg = cx.base + STG_OFF + sb * PSLOT;
+    const uint32_t prow = stg + g * (BM * 128) + (uint32_t)r * 128u;
 #pragma unroll
     for (int q = 0; q < 8; ++q)
-      st_cluster_v4(prow + ((q ^ (r & 7)) << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-    if (g == 0) st_cluster_u32(peer_ctrl + OFF_ALPHA + (sb * BM + r) * 4, __float_as_uint(alpha));
-    fence_proxy_async_cluster();
+      st_shared_v4(prow + ((q ^ (r & 7)) << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    float* stgf = reinterpret_cast<float*>(gbase + STG_OFF + sb * PSLOT);
+    if (g == 0) stgf[(SLOT_ALPHA >> 2) + r] = alpha;
+    fence_proxy_async_cta();
     const bool any = named_bar_red_or(1, GROUP, rescale_row);
     if (threadIdx.x == 64) {
-      st_cluster_u32(peer_ctrl + OFF_FLAG + sb * 4, any ? 1u : 0u);
-      mbar_arrive_remote(peer_ctrl + 8u * P_FULL + 8u * sb);
+      reinterpret_cast<uint32_t*>(stgf)[SLOT_FLAG >> 2] = any ? 1u : 0u;
+      fence_proxy_async_cta();
+      bulk_copy_to_peer(peer_p + sb * PSLOT, stg, SLOT_COPY, peer_ctrl + 8u * P_FULL + 8u * sb);
     }
   }
   // final row statistics for the epilogue: l = both groups' partial sums
@@ -426,9 +431,10 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, uint8_t* gbase, uint32_t t
   uint32_t gi = 0, nres = 0;
   for (int t = 0; t < ntiles && ok; ++t) {
     const uint32_t sb = t & 1;
+    if (lane == 0) mbar_arrive_expect_tx(cx.bar(P_FULL + sb), SLOT_COPY);
     if (!(ok = wait_warp(cx, cx.bar(P_FULL + sb), (t >> 1) & 1, true))) break;
-    fence_proxy_async_cta();
-    const uint32_t flag = ctrl[(OFF_FLAG >> 2) + sb];
+    const uint32_t flag =
+        *reinterpret_cast<volatile uint32_t*>(gbase + P_OFF + sb * PSLOT + SLOT_FLAG);
     if (flag && t > 0) {
       // every earlier PV MMA must be done before O is rescaled
       if (!(ok = wait_warp(cx, cx.bar(PV_TILE), (t - 1) & 1))) break;
@@ -505,7 +511,8 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, uint
     ++nev;
     if (ctrl[OFF_EVTYPE >> 2] != 1u) break;
     const uint32_t sb = ctrl[OFF_EVTILE >> 2];
-    const float a = fctrl[(OFF_ALPHA >> 2) + sb * BM + r];
+    const float a =
+        reinterpret_cast<const volatile float*>(gbase + P_OFF + sb * PSLOT + SLOT_ALPHA)[r];
     tc_fence_after();
     uint32_t v[32];
     for (int c = 0; c < 256 / 32; ++c) {
