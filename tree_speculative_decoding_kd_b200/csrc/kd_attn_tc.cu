@@ -16,15 +16,17 @@
 // The fp32 output accumulator of one M tile (128 x 512) fills all 512 TMEM
 // columns of an SM, leaving none for scores, so each unit of work runs on a
 // 2-CTA cluster with split roles:
-//   rank 0 ("QK" CTA): S = Q K^T into a double-buffered 2 x 128-column TMEM
-//       accumulator.  The eight 64-wide latent chunks of Q sit in the other 256
+//   rank 0 ("QK" CTA): S = Q K^T for 256 keys at a time (M=128, N=256 MMAs, the
+//       shape that keeps the tensor pipe saturated from one issuing thread) into
+//       256 TMEM columns.  The eight 64-wide latent chunks of Q sit in the other 256
 //       TMEM columns and feed the MMA as its A operand from tensor memory; the rope
-//       chunk sits in shared memory.  That leaves shared memory for an 8-stage ring
-//       of 128-key x 64-column K chunks (TMA, 128-byte swizzle) and two P staging
-//       slots.  Two 4-warp softmax groups split each S tile's columns, keep an
-//       online max with a lazy rescale threshold, write bf16 P into a local staging
-//       slot in the K-major swizzled layout the MMA reads, and one thread moves the
-//       slot to rank 1 with a single bulk copy that completes on rank 1's barrier.
+//       chunk sits in shared memory.  Shared memory holds a 4-stage ring of
+//       256-key x 64-column K chunks (TMA, 128-byte swizzle) and two P staging
+//       slots.  Two 4-warp softmax groups copy S into registers (freeing TMEM for
+//       the next tile at once), keep an online max with a lazy rescale threshold,
+//       and emit P as two 128-key halves: each is written into a local staging slot
+//       in the K-major swizzled layout the MMA reads and moved to rank 1 by one
+//       thread with a single bulk copy that completes on rank 1's barrier.
 //   rank 1 ("PV" CTA): O (128 x 512 fp32) in TMEM; V as 64-key x 256-column
 //       groups (four 64-column MN-major boxes) in a 4-deep ring; O += P V as
 //       M=128, N=256, K=16 MMAs; two 4-warp groups apply the rare O rescale and
@@ -57,12 +59,14 @@ using namespace ptx;
 constexpr int NTHREADS = 320;           // warp 0 TMA, warp 1 MMA, warps 2..9 two 4-warp groups
 constexpr int GROUP = 256;              // threads of the two 4-warp groups
 constexpr int BM = 128;                 // query rows per M tile
-constexpr int BN = 128;                 // keys per tile
+constexpr int BQ = 256;                 // keys per QK tile (S = 128 x 256)
+constexpr int BN = 128;                 // keys per P / PV tile (two per QK tile)
 constexpr int KC = 64;                  // columns per 128-byte swizzle atom
 constexpr int NCHUNK = 9;               // 8 latent chunks + 1 rope chunk
 constexpr int CHUNK = BN * KC * 2;      // 16 KB: 128 rows x 64 bf16
+constexpr int KCHUNK = BQ * KC * 2;     // 32 KB: 256 keys x 64 bf16 (one K ring stage)
 constexpr int NQT = 8;                  // Q chunks held in TMEM (the rope chunk in shared memory)
-constexpr int NK = 8;                   // K ring stages
+constexpr int NK = 4;                   // K ring stages
 constexpr int VKEYS = 64;               // keys per V group
 constexpr int VCH = VKEYS * KC * 2;     // 8 KB: 64 keys x 64 latent columns
 constexpr int VG = 4 * VCH;             // one V group: 64 keys x 256 latent columns
@@ -74,7 +78,7 @@ constexpr int SLOT_COPY = PBYTES + 528; // bytes moved to the PV CTA per tile
 constexpr int PSLOT = PBYTES + 1024;    // slot stride (keeps 1024-byte alignment)
 
 // TMEM columns of the QK CTA
-constexpr uint32_t TS = 0;              // S[2]: 2 x 128 columns
+constexpr uint32_t TS = 0;              // S: 256 columns (one 128 x 256 tile)
 constexpr uint32_t TQ = 256;            // Q chunks 0..7: 8 x 32 columns
 
 // control block (same offsets in both CTAs so the peer can address it)
@@ -85,8 +89,8 @@ enum Bar {
   K_FULL = QT_FULL + 1,
   K_EMPTY = K_FULL + NK,
   S_FULL = K_EMPTY + NK,
-  S_EMPTY = S_FULL + 2,
-  P_FREE = S_EMPTY + 2,
+  S_EMPTY = S_FULL + 1,
+  P_FREE = S_EMPTY + 1,
   V_FULL = P_FREE + 2,
   V_EMPTY = V_FULL + NVG,
   P_FULL = V_EMPTY + NVG,
@@ -110,14 +114,14 @@ static_assert(NBAR * 8 <= OFF_TMEM, "barrier block overflow");
 constexpr int Q_OFF = CTRL;                           // Q chunk 8 (rope)
 constexpr int STG_OFF = Q_OFF + (NCHUNK - NQT) * CHUNK; // P staging, 2 slots
 constexpr int K_OFF = STG_OFF + 2 * PSLOT;
-constexpr int QK_END = K_OFF + NK * CHUNK;
+constexpr int QK_END = K_OFF + NK * KCHUNK;
 constexpr int P_OFF = CTRL;
 constexpr int V_OFF = P_OFF + 2 * PSLOT;
 constexpr int PV_END = V_OFF + NVG * VG;
 constexpr int SMEM_BYTES = (QK_END > PV_END ? QK_END : PV_END) + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, 0, 0);    // Q, K both K-major
+constexpr uint32_t IDESC_QK = idesc_bf16(BM, BQ, 0, 0);    // Q, K both K-major
 constexpr uint32_t IDESC_PV = idesc_bf16(BM, 256, 0, 1);   // P K-major, V MN-major
 constexpr float RESCALE_THRESHOLD = 8.0f;                  // log2 units: P <= 2^8
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;          // 2 s per wait
@@ -208,13 +212,13 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const CUtensorMap* tm
   uint32_t it = 0;
   bool ok = true;
   for (int t = 0; t < ntiles && ok; ++t) {
-    const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN);
+    const int32_t krow = (int32_t)(krow0 + (int64_t)t * BQ);
     for (int c = 0; c < NCHUNK; ++c, ++it) {
       const uint32_t st = it % NK, k = it / NK;
       if (!(ok = wait_bar(cx, cx.bar(K_EMPTY + st), (k & 1u) ^ 1u))) break;
-      mbar_arrive_expect_tx(cx.bar(K_FULL + st), CHUNK);
-      if (c < 8) tma_load_2d(base + K_OFF + st * CHUNK, tm_c, c * KC, krow, cx.bar(K_FULL + st));
-      else tma_load_2d(base + K_OFF + st * CHUNK, tm_r, 0, krow, cx.bar(K_FULL + st));
+      mbar_arrive_expect_tx(cx.bar(K_FULL + st), KCHUNK);
+      if (c < 8) tma_load_2d(base + K_OFF + st * KCHUNK, tm_c, c * KC, krow, cx.bar(K_FULL + st));
+      else tma_load_2d(base + K_OFF + st * KCHUNK, tm_r, 0, krow, cx.bar(K_FULL + st));
     }
   }
   // every armed stage must have landed before the CTA may exit
@@ -230,15 +234,14 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, uint32_t tmem, int ntiles)
   tc_fence_after();
   uint32_t it = 0;
   for (int t = 0; t < ntiles && ok; ++t) {
-    const uint32_t sb = t & 1;
-    if (!(ok = wait_bar(cx, cx.bar(S_EMPTY + sb), ((t >> 1) & 1) ^ 1))) break;
+    if (!(ok = wait_bar(cx, cx.bar(S_EMPTY), (t & 1) ^ 1))) break;
     tc_fence_after();
-    const uint32_t d = tmem + TS + sb * BN;
+    const uint32_t d = tmem + TS;
     for (int c = 0; c < NCHUNK; ++c, ++it) {
       const uint32_t st = it % NK;
       if (!(ok = wait_bar(cx, cx.bar(K_FULL + st), (it / NK) & 1u))) break;
       tc_fence_after();
-      const uint32_t b0 = base + K_OFF + st * CHUNK;
+      const uint32_t b0 = base + K_OFF + st * KCHUNK;
       if (c < NQT) {
 #pragma unroll
         for (int kk = 0; kk < KC / 16; ++kk)
@@ -251,10 +254,45 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, uint32_t tmem, int ntiles)
       }
       tc_commit(cx.bar(K_EMPTY + st));
     }
-    if (ok) tc_commit(cx.bar(S_FULL + sb));
+    if (ok) tc_commit(cx.bar(S_FULL));
   }
   tc_commit(cx.bar(DRAIN));
   wait_bar(cx, cx.bar(DRAIN), 0);
+}
+
+// One 128-key half of a QK tile: exponentiate this thread's 64 columns against
+// the row reference mb, add them to the running sum, and ship the bf16 P tile
+// (plus the per-row rescale factor for the PV side) through staging slot u % 2.
+__device__ __forceinline__ bool emit_p(const Ctx& cx, uint8_t* gbase, const float (&x)[64], int u,
+                                       float mb, float alpha, bool rescale_row, int r, int g,
+                                       uint32_t peer_p, uint32_t peer_ctrl, float& l_part) {
+  const uint32_t sb = u & 1;
+  float rs[4] = {0.f, 0.f, 0.f, 0.f};
+  uint32_t pk[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const float p0 = ex2(x[2 * c] - mb), p1 = ex2(x[2 * c + 1] - mb);
+    rs[c & 3] += p0 + p1;
+    pk[c] = pack_bf16x2(p0, p1);
+  }
+  l_part += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+  // staging slot sb (and the peer's P slot sb) is free once the PV MMAs of P tile u-2 completed
+  if (!wait_group(cx, cx.bar(P_FREE + sb), ((u >> 1) & 1) ^ 1)) return false;
+  const uint32_t stg = cx.base + STG_OFF + sb * PSLOT;
+  const uint32_t prow = stg + g * (BM * 128) + (uint32_t)r * 128u;
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    st_shared_v4(prow + ((q ^ (r & 7)) << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+  float* stgf = reinterpret_cast<float*>(gbase + STG_OFF + sb * PSLOT);
+  if (g == 0) stgf[(SLOT_ALPHA >> 2) + r] = alpha;
+  fence_proxy_async_cta();
+  const bool any = named_bar_red_or(1, GROUP, rescale_row);
+  if (threadIdx.x == 64) {
+    reinterpret_cast<uint32_t*>(stgf)[SLOT_FLAG >> 2] = any ? 1u : 0u;
+    fence_proxy_async_cta();
+    bulk_copy_to_peer(peer_p + sb * PSLOT, stg, SLOT_COPY, peer_ctrl + 8u * P_FULL + 8u * sb);
+  }
+  return true;
 }
 
 // Softmax groups: thread (g, r) owns row r and key columns [64 g, 64 g + 64) of every tile.
@@ -307,40 +345,50 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
   float m_ref = -INFINITY, l_part = 0.f;
   bool ok = true;
   for (int t = 0; t < ntiles && ok; ++t) {
-    const uint32_t sb = t & 1;
-    if (!(ok = wait_group(cx, cx.bar(S_FULL + sb), (t >> 1) & 1))) break;
+    if (!(ok = wait_group(cx, cx.bar(S_FULL), t & 1))) break;
     tc_fence_after();
-    float x[64];
+    // this thread's columns: keys 64 g .. 64 g + 63 of each 128-key half h of the tile
+    float x[2][64];
     {
-      uint32_t u0[32], u1[32];
-      tmem_ld32(lane_addr + TS + sb * BN + g * 64, u0);
-      tmem_ld32(lane_addr + TS + sb * BN + g * 64 + 32, u1);
+      uint32_t u[4][32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        tmem_ld32(lane_addr + TS + h * BN + g * 64, u[2 * h]);
+        tmem_ld32(lane_addr + TS + h * BN + g * 64 + 32, u[2 * h + 1]);
+      }
       tmem_wait_ld();
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        x[k] = __uint_as_float(u0[k]) * p.scale_log2;
-        x[32 + k] = __uint_as_float(u1[k]) * p.scale_log2;
-      }
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          x[h][k] = __uint_as_float(u[2 * h][k]) * p.scale_log2;
+          x[h][32 + k] = __uint_as_float(u[2 * h + 1][k]) * p.scale_log2;
+        }
     }
     tc_fence_before();
-    mbar_arrive(cx.bar(S_EMPTY + sb));
+    mbar_arrive(cx.bar(S_EMPTY));              // TMEM free for the next tile's MMAs
     // mask: only keys at or beyond L need it
-    const int64_t kt = kbeg + (int64_t)t * BN + g * 64;
-    if (kt + 64 > L) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const int64_t k = kt + c - L;
-        bool vis_c = true;
-        if (k >= 0) vis_c = (k < n) && ((mask_word(w, (int)k >> 5) >> ((int)k & 31)) & 1u);
-        if (!vis_c) x[c] = -INFINITY;
+    for (int h = 0; h < 2; ++h) {
+      const int64_t kt = kbeg + (int64_t)t * BQ + h * BN + g * 64;
+      if (kt + 64 > L) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int64_t k = kt + c - L;
+          bool vis_c = true;
+          if (k >= 0) vis_c = (k < n) && ((mask_word(w, (int)k >> 5) >> ((int)k & 31)) & 1u);
+          if (!vis_c) x[h][c] = -INFINITY;
+        }
       }
     }
-    float mx[4] = {x[0], x[1], x[2], x[3]};
+    float mx[4] = {x[0][0], x[0][1], x[0][2], x[0][3]};
 #pragma unroll
-    for (int c = 4; c < 64; c += 4) {
-      mx[0] = fmaxf(mx[0], x[c]); mx[1] = fmaxf(mx[1], x[c + 1]);
-      mx[2] = fmaxf(mx[2], x[c + 2]); mx[3] = fmaxf(mx[3], x[c + 3]);
-    }
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int c = (h == 0 ? 4 : 0); c < 64; c += 4) {
+        mx[0] = fmaxf(mx[0], x[h][c]); mx[1] = fmaxf(mx[1], x[h][c + 1]);
+        mx[2] = fmaxf(mx[2], x[h][c + 2]); mx[3] = fmaxf(mx[3], x[h][c + 3]);
+      }
     xch[g * BM + r] = max4(mx[0], mx[1], mx[2], mx[3]);
     named_bar_sync(1, GROUP);
     const float tmax = fmaxf(xch[r], xch[BM + r]);
@@ -357,31 +405,8 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
       m_ref = tmax;
     }
     const float mb = m_ref == -INFINITY ? 0.f : m_ref;
-    float rs[4] = {0.f, 0.f, 0.f, 0.f};
-    uint32_t pk[32];
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const float p0 = ex2(x[2 * c] - mb), p1 = ex2(x[2 * c + 1] - mb);
-      rs[c & 3] += p0 + p1;
-      pk[c] = pack_bf16x2(p0, p1);
-    }
-    l_part += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-    // staging slot sb (and the peer's P slot sb) is free once the PV MMAs of tile t-2 completed
-    if (!(ok = wait_group(cx, cx.bar(P_FREE + sb), ((t >> 1) & 1) ^ 1))) break;
-    const uint32_t stg = cx.base + STG_OFF + sb * PSLOT;
-    const uint32_t prow = stg + g * (BM * 128) + (uint32_t)r * 128u;
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      st_shared_v4(prow + ((q ^ (r & 7)) << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-    float* stgf = reinterpret_cast<float*>(gbase + STG_OFF + sb * PSLOT);
-    if (g == 0) stgf[(SLOT_ALPHA >> 2) + r] = alpha;
-    fence_proxy_async_cta();
-    const bool any = named_bar_red_or(1, GROUP, rescale_row);
-    if (threadIdx.x == 64) {
-      reinterpret_cast<uint32_t*>(stgf)[SLOT_FLAG >> 2] = any ? 1u : 0u;
-      fence_proxy_async_cta();
-      bulk_copy_to_peer(peer_p + sb * PSLOT, stg, SLOT_COPY, peer_ctrl + 8u * P_FULL + 8u * sb);
-    }
+    ok = emit_p(cx, gbase, x[0], 2 * t, mb, alpha, rescale_row, r, g, peer_p, peer_ctrl, l_part) &&
+         emit_p(cx, gbase, x[1], 2 * t + 1, mb, 1.f, false, r, g, peer_p, peer_ctrl, l_part);
   }
   // final row statistics for the epilogue: l = both groups' partial sums
   named_bar_sync(1, GROUP);
@@ -395,9 +420,10 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
   if (threadIdx.x == 64) {
     mbar_arrive_remote(peer_ctrl + 8u * STATS);
     // the last P_FREE arrivals come from the peer's MMA completion: wait for them
+    const int np = 2 * ntiles;
     if (ok)
-      for (int t = (ntiles > 2 ? ntiles - 2 : 0); t < ntiles; ++t)
-        wait_bar(cx, cx.bar(P_FREE + (t & 1)), (t >> 1) & 1);
+      for (int u = (np > 2 ? np - 2 : 0); u < np; ++u)
+        wait_bar(cx, cx.bar(P_FREE + (u & 1)), (u >> 1) & 1);
   }
 }
 
@@ -406,7 +432,7 @@ __device__ __forceinline__ void pv_producer(const Ctx& cx, const CUtensorMap* tm
                                             int ntiles) {
   bool ok = true;
   uint32_t gi = 0;
-  for (int t = 0; t < ntiles && ok; ++t) {
+  for (int t = 0; t < 2 * ntiles && ok; ++t) {
     for (int kh = 0; kh < BN / VKEYS && ok; ++kh) {
       const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN + kh * VKEYS);
       for (int hh = 0; hh < 2; ++hh, ++gi) {
@@ -429,7 +455,7 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, uint8_t* gbase, uint32_t t
   volatile uint32_t* ctrl = reinterpret_cast<volatile uint32_t*>(gbase);
   bool ok = true;
   uint32_t gi = 0, nres = 0;
-  for (int t = 0; t < ntiles && ok; ++t) {
+  for (int t = 0; t < 2 * ntiles && ok; ++t) {      // P tiles of 128 keys
     const uint32_t sb = t & 1;
     if (lane == 0) mbar_arrive_expect_tx(cx.bar(P_FULL + sb), SLOT_COPY);
     if (!(ok = wait_warp(cx, cx.bar(P_FULL + sb), (t >> 1) & 1, true))) break;
@@ -585,7 +611,7 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, uint
 }
 
 // ====================================================================== kernel
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(200)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant__ CUtensorMap tm_qr,
                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
@@ -608,10 +634,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
     return;
   }
   const int64_t nkeys = L + n;
-  const int T = (int)((nkeys + BN - 1) / BN);
+  const int T = (int)((nkeys + BQ - 1) / BQ);         // 256-key QK tiles
   const int t0 = (int)((int64_t)sp * T / p.splits), t1 = (int)((int64_t)(sp + 1) * T / p.splits);
   const int ntiles = t1 - t0;
-  const int64_t kbeg = (int64_t)t0 * BN;                    // request-relative first key
+  const int64_t kbeg = (int64_t)t0 * BQ;                    // request-relative first key
   const int64_t krow0 = (int64_t)b * p.cap + kbeg;          // cache row of the first key
   const int qrow0 = b * n * H + mt * BM;
 
@@ -624,7 +650,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
       uint32_t cnt = 1;
-      if (i == QT_FULL || i == S_EMPTY || i == S_EMPTY + 1 || i == CORR_DONE) cnt = GROUP;
+      if (i == QT_FULL || i == S_EMPTY || i == CORR_DONE) cnt = GROUP;
       mbar_init(cx.bar(i), cnt);
     }
     *cx.abort_flag = 0u;
@@ -739,7 +765,7 @@ static int active_pairs(int sms) {
 int auto_splits(int B, int n, int H, int64_t cap, int pairs) {
   const int64_t mtiles = ((int64_t)n * H + tc::BM - 1) / tc::BM;
   const int64_t units = (int64_t)B * mtiles;
-  const int64_t T = (cap + tc::BN - 1) / tc::BN;
+  const int64_t T = (cap + tc::BQ - 1) / tc::BQ;
   int best = 1;
   double best_cost = 1e300;
   for (int s = 1; s <= 64 && s <= T; ++s) {
@@ -807,8 +833,8 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   CUtensorMap tq, tr, tcv, tkr, tv;
   if ((st = tc::make_map(&tq, q_abs, KD_D_C, (uint64_t)rows, KD_D_C * 2, tc::BM))) return st;
   if ((st = tc::make_map(&tr, q_rope, KD_D_R, (uint64_t)rows, KD_D_R * 2, tc::BM))) return st;
-  if ((st = tc::make_map(&tcv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::BN))) return st;
-  if ((st = tc::make_map(&tkr, k_rope, KD_D_R, (uint64_t)(B * cap), (uint64_t)sr * 2, tc::BN))) return st;
+  if ((st = tc::make_map(&tcv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::BQ))) return st;
+  if ((st = tc::make_map(&tkr, k_rope, KD_D_R, (uint64_t)(B * cap), (uint64_t)sr * 2, tc::BQ))) return st;
   if ((st = tc::make_map(&tv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::VKEYS))) return st;
 
   tc::Params prm;
