@@ -611,7 +611,7 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, uint
 }
 
 // ====================================================================== kernel
-__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(200)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant__ CUtensorMap tm_qr,
                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
