@@ -130,7 +130,6 @@ struct Params {
   const int32_t* cache_lens;
   const uint32_t* vis;
   const int32_t* positions;
-  const uint16_t* q_abs;
   uint16_t* out;
   float* lse;
   float* part_o;
@@ -184,6 +183,12 @@ __device__ __forceinline__ bool wait_group(const Ctx& cx, uint32_t bar, uint32_t
   return !named_bar_red_or(1, GROUP, !ok);
 }
 
+// Shared-memory offset where TMA drops Q latent chunk c (0..7) at the start of a unit.
+__host__ __device__ constexpr int q_stage_off(int c) {
+  return c < 4 ? STG_OFF + c * CHUNK : K_OFF + 2 * KCHUNK + (c - 4) * CHUNK;
+}
+static_assert(4 * CHUNK <= 2 * PSLOT && 2 * KCHUNK + 4 * CHUNK <= NK * KCHUNK, "Q landing zones");
+
 __device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {      // K-major, SW128
   return smem_desc_sw128(saddr, 16, 1024);
 }
@@ -207,7 +212,10 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const CUtensorMap* tm
                                             const CUtensorMap* tm_r, int qrow0, int64_t krow0,
                                             int ntiles) {
   const uint32_t base = cx.base;
-  mbar_arrive_expect_tx(cx.bar(Q_FULL), (NCHUNK - NQT) * CHUNK);
+  // Q: latent chunks 0..3 land in the (still unused) P staging area, chunks 4..7 in
+  // K ring stages 2..3; the softmax groups move them into TMEM.  The rope chunk stays.
+  mbar_arrive_expect_tx(cx.bar(Q_FULL), NCHUNK * CHUNK);
+  for (int c = 0; c < NQT; ++c) tma_load_2d(base + q_stage_off(c), tm_qa, c * KC, qrow0, cx.bar(Q_FULL));
   tma_load_2d(base + Q_OFF, tm_qr, 0, qrow0, cx.bar(Q_FULL));
   uint32_t it = 0;
   bool ok = true;
@@ -216,6 +224,7 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const CUtensorMap* tm
     for (int c = 0; c < NCHUNK; ++c, ++it) {
       const uint32_t st = it % NK, k = it / NK;
       if (!(ok = wait_bar(cx, cx.bar(K_EMPTY + st), (k & 1u) ^ 1u))) break;
+      if (it == 2 && !(ok = wait_bar(cx, cx.bar(QT_FULL), 0))) break;   // stages 2, 3 held Q
       mbar_arrive_expect_tx(cx.bar(K_FULL + st), KCHUNK);
       if (c < 8) tma_load_2d(base + K_OFF + st * KCHUNK, tm_c, c * KC, krow, cx.bar(K_FULL + st));
       else tma_load_2d(base + K_OFF + st * KCHUNK, tm_r, 0, krow, cx.bar(K_FULL + st));
@@ -310,22 +319,25 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
   const int node = valid ? R / H : 0;
   float* xch = reinterpret_cast<float*>(gbase + OFF_XCH);
 
-  // ---- Q chunks 0..7 of this row into TMEM (group 0: chunks 0..3, group 1: 4..7)
+  // ---- Q chunks 0..7 of this row into TMEM (group 0: chunks 0..3, group 1: 4..7),
+  //      read back from the 128-byte-swizzled TMA landing zones
   {
-    const int64_t grow = (int64_t)b * rows_req + R;
-    const bool in_range = R < rows_req;
-    const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + grow * KD_D_C);
-    const int c0 = g * 4, c1 = g * 4 + 4;
-    for (int c = c0; c < c1; ++c) {
-      uint32_t v[32];
+    const bool okq = wait_group(cx, cx.bar(Q_FULL), 0);
+    if (okq) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint4 x = in_range ? src[c * 8 + q] : make_uint4(0u, 0u, 0u, 0u);
-        v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const int c = g * 4 + c4;
+        const uint8_t* row = gbase + q_stage_off(c) + r * 128;
+        uint32_t v[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint4 x = *reinterpret_cast<const uint4*>(row + ((q ^ (r & 7)) << 4));
+          v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+        }
+        tmem_st32(lane_addr + TQ + c * 32, v);
       }
-      tmem_st32(lane_addr + TQ + c * 32, v);
+      tmem_wait_st();
     }
-    tmem_wait_st();
     tc_fence_before();
     mbar_arrive(cx.bar(QT_FULL));
   }
@@ -350,20 +362,15 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
     // this thread's columns: keys 64 g .. 64 g + 63 of each 128-key half h of the tile
     float x[2][64];
     {
-      uint32_t u[4][32];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        tmem_ld32(lane_addr + TS + h * BN + g * 64, u[2 * h]);
-        tmem_ld32(lane_addr + TS + h * BN + g * 64 + 32, u[2 * h + 1]);
-      }
+      uint32_t u0[64], u1[64];
+      tmem_ld64(lane_addr + TS + g * 64, u0);
+      tmem_ld64(lane_addr + TS + BN + g * 64, u1);
       tmem_wait_ld();
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          x[h][k] = __uint_as_float(u[2 * h][k]) * p.scale_log2;
-          x[h][32 + k] = __uint_as_float(u[2 * h + 1][k]) * p.scale_log2;
-        }
+      for (int k = 0; k < 64; ++k) {
+        x[0][k] = __uint_as_float(u0[k]) * p.scale_log2;
+        x[1][k] = __uint_as_float(u1[k]) * p.scale_log2;
+      }
     }
     tc_fence_before();
     mbar_arrive(cx.bar(S_EMPTY));              // TMEM free for the next tile's MMAs
@@ -521,8 +528,9 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, uint8_t* gbase, uint32_t t
 }
 
 // Correction / epilogue groups: thread (g, r) owns row r, O columns [256 g, 256 g + 256).
-__device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, uint8_t* gbase,
-                                            uint32_t tmem, int b, int mt, int sp, int ntiles) {
+__device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, const CUtensorMap* tm_o,
+                                            uint8_t* gbase, uint32_t tmem, int b, int mt, int sp,
+                                            int ntiles) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = (warp - 2) >> 2;
   const int quad = warp & 3;
@@ -564,33 +572,48 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, uint
   const bool have_o = ntiles > 0;
   const int64_t grow = (int64_t)b * rows_req + R;
   const int64_t prow = ((int64_t)sp * p.B * rows_req) + grow;
-  uint32_t v0[32], v1[32];
-  for (int c = 0; c < 256 / 64; ++c) {
-    if (have_o && ok) {
-      tmem_ld32(lane_addr + c * 64, v0);
-      tmem_ld32(lane_addr + c * 64 + 32, v1);
-      tmem_wait_ld();
-    } else {
+  if (p.splits == 1) {
+    // bf16 tile -> eight 128-row x 64-column boxes in the (now idle) V ring, laid out
+    // with the 128-byte swizzle, then TMA stores; the per-request 3-D tensor map
+    // clips rows past the request's last node.
+    for (int c = 0; c < 256 / 64; ++c) {
+      uint32_t v[64];
+      if (have_o && ok) {
+        tmem_ld64(lane_addr + c * 64, v);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-      for (int k = 0; k < 32; ++k) v0[k] = v1[k] = 0u;
-    }
-    if (!valid) continue;
-    const int col = g * 256 + c * 64;
-    if (p.splits == 1) {
-      uint4* dst = reinterpret_cast<uint4*>(p.out + grow * KD_D_C + col);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int o = q * 8;
-        dst[q] = make_uint4(pack_bf16x2(__uint_as_float(v0[o + 0]) * inv, __uint_as_float(v0[o + 1]) * inv),
-                            pack_bf16x2(__uint_as_float(v0[o + 2]) * inv, __uint_as_float(v0[o + 3]) * inv),
-                            pack_bf16x2(__uint_as_float(v0[o + 4]) * inv, __uint_as_float(v0[o + 5]) * inv),
-                            pack_bf16x2(__uint_as_float(v0[o + 6]) * inv, __uint_as_float(v0[o + 7]) * inv));
-        dst[4 + q] = make_uint4(pack_bf16x2(__uint_as_float(v1[o + 0]) * inv, __uint_as_float(v1[o + 1]) * inv),
-                                pack_bf16x2(__uint_as_float(v1[o + 2]) * inv, __uint_as_float(v1[o + 3]) * inv),
-                                pack_bf16x2(__uint_as_float(v1[o + 4]) * inv, __uint_as_float(v1[o + 5]) * inv),
-                                pack_bf16x2(__uint_as_float(v1[o + 6]) * inv, __uint_as_float(v1[o + 7]) * inv));
+        for (int k = 0; k < 64; ++k) v[k] = 0u;
       }
-    } else {
+      const uint32_t box = cx.base + V_OFF + (g * 4 + c) * CHUNK + (uint32_t)r * 128u;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        st_shared_v4(box + ((q ^ (r & 7)) << 4),
+                     pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv),
+                     pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv),
+                     pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv),
+                     pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv));
+    }
+    fence_proxy_async_cta();
+    named_bar_sync(1, GROUP);
+    if (threadIdx.x == 64 && ok) {
+      for (int bx = 0; bx < 8; ++bx) tma_store_3d(tm_o, cx.base + V_OFF + bx * CHUNK, bx * KC, mt * BM, b);
+      bulk_commit_group();
+      bulk_wait_group_read0();
+    }
+  } else {
+    uint32_t v0[32], v1[32];
+    for (int c = 0; c < 256 / 64; ++c) {
+      if (have_o && ok) {
+        tmem_ld32(lane_addr + c * 64, v0);
+        tmem_ld32(lane_addr + c * 64 + 32, v1);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v0[k] = v1[k] = 0u;
+      }
+      if (!valid) continue;
+      const int col = g * 256 + c * 64;
       float4* dst = reinterpret_cast<float4*>(p.part_o + prow * KD_D_C + col);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
@@ -614,7 +637,8 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, uint
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant__ CUtensorMap tm_qr,
                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -666,6 +690,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
     tma_prefetch_desc(&tm_c);
     tma_prefetch_desc(&tm_r);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
   }
   tc_fence_before();
   cluster_sync();
@@ -687,7 +712,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
     } else if (warp == 1) {
       pv_mma(cx, gbase, tmem, kbeg, nkeys, ntiles);
     } else {
-      pv_epilogue(cx, p, gbase, tmem, b, mt, sp, ntiles);
+      pv_epilogue(cx, p, &tm_o, gbase, tmem, b, mt, sp, ntiles);
     }
   }
 
@@ -727,6 +752,24 @@ static int make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t ro
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+    return KD_ELAUNCH;
+  }
+  return KD_OK;
+}
+
+// Per-request 3-D bf16 view [B][rows][512] of the output, 64 x 128 x 1 boxes, 128-byte swizzle.
+static int make_out_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t B) {
+  auto fn = encode_fn();
+  if (!fn) return KD_ELAUNCH;
+  cuuint64_t dims[3] = {KD_D_C, rows, B};
+  cuuint64_t strides[2] = {KD_D_C * 2, rows * KD_D_C * 2};
+  cuuint32_t box[3] = {KC, BM, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled(out)");
     return KD_ELAUNCH;
   }
   return KD_OK;
@@ -830,18 +873,18 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   }
   if (workspace_bytes_for(B, n, H, splits) > ws_bytes) return KD_ERANGE;
 
-  CUtensorMap tq, tr, tcv, tkr, tv;
+  CUtensorMap tq, tr, tcv, tkr, tv, to;
   if ((st = tc::make_map(&tq, q_abs, KD_D_C, (uint64_t)rows, KD_D_C * 2, tc::BM))) return st;
   if ((st = tc::make_map(&tr, q_rope, KD_D_R, (uint64_t)rows, KD_D_R * 2, tc::BM))) return st;
   if ((st = tc::make_map(&tcv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::BQ))) return st;
   if ((st = tc::make_map(&tkr, k_rope, KD_D_R, (uint64_t)(B * cap), (uint64_t)sr * 2, tc::BQ))) return st;
   if ((st = tc::make_map(&tv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::VKEYS))) return st;
+  if ((st = tc::make_out_map(&to, out, (uint64_t)rows / B, (uint64_t)B))) return st;
 
   tc::Params prm;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   prm.cache_lens = cache_lens;
   prm.vis = vis;
-  prm.q_abs = q_abs;
   prm.positions = positions;
   prm.out = out;
   prm.lse = lse;
@@ -859,7 +902,7 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   prm.scale_log2 = scale * 1.4426950408889634f;
   const int64_t units = (int64_t)B * prm.mtiles * splits;
   if (2 * units > INT32_MAX) return KD_EINVAL;
-  tc::attn_tc_kernel<<<dim3((unsigned)(2 * units)), tc::NTHREADS, tc::SMEM_BYTES, stream>>>(tq, tr, tcv, tkr, tv,
+  tc::attn_tc_kernel<<<dim3((unsigned)(2 * units)), tc::NTHREADS, tc::SMEM_BYTES, stream>>>(tq, tr, tcv, tkr, tv, to,
                                                                                          prm);
   st = launch_status("attn_tc_kernel");
   if (st || splits == 1) return st;
