@@ -322,7 +322,8 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
   // ---- Q chunks 0..7 of this row into TMEM (group 0: chunks 0..3, group 1: 4..7),
   //      read back from the 128-byte-swizzled TMA landing zones
   {
-    const bool okq = wait_group(cx, cx.bar(Q_FULL), 0);
+    // an empty key partition issues no loads at all (its producer does not run)
+    const bool okq = ntiles > 0 && wait_group(cx, cx.bar(Q_FULL), 0);
     if (okq) {
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
