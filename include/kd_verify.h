@@ -150,6 +150,39 @@ int kd_tree_verify_attn_simt(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* 
                              cudaStream_t stream);
 
 /*
+ * kd_tree_verify_attn_noalloc -- kd_tree_verify_attn for callers that cannot
+ * allocate device memory at call time: code running under CUDA graph capture,
+ * serving loops that keep allocator calls off the hot path, and C hosts without a
+ * device allocator.  (The pages have no counterpart; this is an interface
+ * convenience of this library.)
+ *
+ * Same inputs, outputs and checks as kd_tree_verify_attn, without the workspace
+ * arguments.  The workspace is a fixed array of KD_NOALLOC_SCRATCH_BYTES inside the
+ * library; every GPU that loads the library holds it until the process exits.
+ *   - With kv_splits = 0 the split count is chosen so that the partials fit the
+ *     array; an explicit kv_splits whose workspace would exceed it returns KD_ERANGE
+ *     and enqueues nothing.
+ *   - The call allocates nothing: no cudaMalloc/cudaFree and no allocating library
+ *     routine.  It enqueues a 4-byte memset of the array's error word, the attention
+ *     kernels and, when dev_error is not NULL, a 4-byte device-to-device copy of this
+ *     call's KD_DEV_* bits into *dev_error (which is overwritten, not ORed).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and sets kernel attributes; make that first call before
+ *     any stream capture.
+ *   - All calls share the one array and it keeps the previous call's contents: calls
+ *     whose kernels overlap on the GPU (e.g. on two streams without ordering between
+ *     them) race on it and must be serialised by the caller.
+ */
+#define KD_NOALLOC_SCRATCH_BYTES (32 << 20)
+int kd_tree_verify_attn_noalloc(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* q_rope,
+                                const kd_bf16_t* c_kv, const kd_bf16_t* k_rope,
+                                int64_t kv_row_stride_c, int64_t kv_row_stride_r, int64_t cap,
+                                const int32_t* cache_lens, const uint32_t* vis,
+                                const int32_t* positions, int B, int n, int H, float scale,
+                                kd_bf16_t* out, float* lse, int kv_splits, int32_t* dev_error,
+                                cudaStream_t stream);
+
+/*
  * kd_tree_accept -- greedy acceptance of B verified trees.
  *   node_tokens [B][n], parents [B][n], target_argmax [B][n] int32 (target_argmax[b][i]
  *   is the target's prediction after node i).

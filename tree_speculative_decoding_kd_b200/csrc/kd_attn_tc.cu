@@ -909,3 +909,57 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   if (st || splits == 1) return st;
   return launch_combine(prm.part_o, prm.part_lse, cache_lens, B, n, H, cap, splits, out, lse, stream);
 }
+
+// ================================================================== allocation-free variant
+// Some callers cannot allocate device memory when they verify: code running while
+// a CUDA graph is being captured (allocation calls are not allowed there), serving
+// loops that forbid allocator traffic on the hot path, and C hosts that embed this
+// library without a device allocator of their own.  They use the entry point below,
+// which takes its workspace from a fixed array that lives in this library instead
+// of from the caller.  The array is KD_NOALLOC_SCRATCH_BYTES large and every GPU
+// that loads the library keeps it until the process exits.
+namespace kd {
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KD_NOALLOC_SCRATCH_BYTES];
+}  // namespace kd
+
+extern "C" int kd_tree_verify_attn_noalloc(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* q_rope,
+                                           const kd_bf16_t* c_kv, const kd_bf16_t* k_rope,
+                                           int64_t kv_row_stride_c, int64_t kv_row_stride_r,
+                                           int64_t cap, const int32_t* cache_lens,
+                                           const uint32_t* vis, const int32_t* positions, int B,
+                                           int n, int H, float scale, kd_bf16_t* out, float* lse,
+                                           int kv_splits, int32_t* dev_error, cudaStream_t stream) {
+  // Requests that need more split-KV scratch than the array holds are refused here;
+  // with kv_splits = 0 the automatic policy picks a split count that fits.
+  if (kv_splits < 0 || kv_splits > 64) return KD_EINVAL;
+  if (kv_splits > 0) {
+    const size_t need = kd_verify_workspace_bytes(B, n, H, cap, kv_splits);
+    if (need == 0) return KD_EINVAL;
+    if (need > (size_t)KD_NOALLOC_SCRATCH_BYTES) return KD_ERANGE;
+  }
+  // Host code sees the array's name only as a stand-in, so the device address is
+  // looked up once per device, with that device current, on the first call.
+  static void* scratch_ptr[64];
+  int dev = 0;
+  int st = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st) return st;
+  if (dev < 0 || dev >= 64) return KD_ENODEV;
+  if (!scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    st = cuda_status(cudaGetSymbolAddress(&ptr, kd::g_noalloc_scratch), "cudaGetSymbolAddress");
+    if (st) return st;
+    scratch_ptr[dev] = ptr;
+  }
+  void* scratch = scratch_ptr[dev];
+  int32_t* err_word = static_cast<int32_t*>(scratch);   // first int32 of the workspace
+  st = cuda_status(cudaMemsetAsync(err_word, 0, sizeof(int32_t), stream), "cudaMemsetAsync(error word)");
+  if (st) return st;
+  st = kd_tree_verify_attn(q_nope_absorbed, q_rope, c_kv, k_rope, kv_row_stride_c, kv_row_stride_r, cap,
+                           cache_lens, vis, positions, B, n, H, scale, out, lse, scratch,
+                           (size_t)KD_NOALLOC_SCRATCH_BYTES, kv_splits, stream);
+  if (st) return st;
+  if (dev_error)
+    st = cuda_status(cudaMemcpyAsync(dev_error, err_word, sizeof(int32_t), cudaMemcpyDeviceToDevice, stream),
+                     "cudaMemcpyAsync(error word)");
+  return st;
+}

@@ -34,6 +34,8 @@ _SIGS = {
                                  _p, _p, _p, _sz, _i, _p]),
     "kd_tree_verify_attn_simt": (_i, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i,
                                       _f, _p, _p, _p, _p]),
+    "kd_tree_verify_attn_noalloc": (_i, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i,
+                                         _f, _p, _p, _i, _p, _p]),
     "kd_tree_accept": (_i, [_p, _p, _p, _i, _i, _p, _p, _p, _p, _p]),
     "kd_kv_compact": (_i, [_p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _p, _p]),
     "kd_kv_write_nodes": (_i, [_p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _p, _p]),
@@ -152,6 +154,20 @@ def kd_tree_verify_attn(q_abs, q_rope, c_kv, k_rope, cache_lens, vis, positions=
                                    float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), int(kv_splits),
                                    _stream(stream)), "kd_tree_verify_attn")
+    return out, lse
+
+
+def kd_tree_verify_attn_noalloc(q_abs, q_rope, c_kv, k_rope, cache_lens, vis, positions=None,
+                                scale=1.0 / math.sqrt(192.0), out=None, lse=None, kv_splits=0,
+                                dev_error=None, stream=None):
+    """kd_tree_verify_attn with the library's fixed workspace (no allocation by the call)."""
+    B, n, H, sc, sr, cap, out, lse = _attn_args(q_abs, q_rope, c_kv, k_rope, cache_lens, vis,
+                                                positions, out, lse)
+    _check(lib.kd_tree_verify_attn_noalloc(_ptr(q_abs), _ptr(q_rope), _ptr(c_kv), _ptr(k_rope), sc,
+                                           sr, cap, _ptr(cache_lens), _ptr(vis), _ptr(positions),
+                                           B, n, H, float(scale), _ptr(out), _ptr(lse),
+                                           int(kv_splits), _ptr(dev_error), _stream(stream)),
+           "kd_tree_verify_attn_noalloc")
     return out, lse
 
 
