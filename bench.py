@@ -33,6 +33,23 @@ METRIC = "tree-verify MLA attn TFLOP/s + KV HBM GB/s (% roofline); verify steps/
 N_DISTINCT = 8          # distinct pre-generated step inputs, cycled
 
 
+def profiled_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, only while the
+    attention kernel source is the one those counters were taken from (else None)."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "verify_step_loop_launch_list.md")
+    src = os.path.join(ROOT, "tree_speculative_decoding_kd_b200", "csrc", "kd_attn_tc.cu")
+    try:
+        text = open(prof).read()
+        want = text.split("kernel_source_sha256_16:")[1].split()[0]
+        have = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if want != have:
+            return None
+        return int(text.split("traffic_bytes_per_launch:")[1].split()[0])
+    except (OSError, IndexError, ValueError):
+        return None
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -356,7 +373,10 @@ def run_kd(args):
         achieved = flop_avg / attn_avg / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": None,
+                "traffic": profiled_traffic(),
+                "traffic_source": "ncu dram__bytes_read+write of one launch of this workload "
+                                  "(profiles/verify_step_loop_launch_list.md); null if the kernel "
+                                  "changed since",
                 "peak_source": f"{peaks['source']} bf16 burst (cuBLAS)",
                 "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
                 "kernel": "attn_tc_kernel (tree-verify attention)",
