@@ -203,18 +203,16 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) {     // MN-major, S
 // 2^f, and n added to the result's exponent field.  The cubic is the
 // relative-error minimax fit of 2^f on [-1/2, 1/2] found by a Remez exchange:
 // max relative error 7.5e-5 (also when evaluated in fp32), far below the bf16
-// rounding that P undergoes next.  The arithmetic runs on y clamped at -126 (so
-// that the exponent sum never leaves the normal range: 2^f < 1 carries exponent
-// field 126), and any y below -126 -- a masked key is -inf -- returns exactly 0.
+// rounding that P undergoes next.  y is clamped at -127 so that -inf (a masked
+// key) gives exactly 0.
 __device__ __forceinline__ float exp2_fma(float y) {
-  const float yc = fmaxf(y, -126.f);
-  const float t = yc + 12582912.f;
-  const float f = yc - (t - 12582912.f);
+  y = fmaxf(y, -127.f);
+  const float t = y + 12582912.f;
+  const float f = y - (t - 12582912.f);
   float q = fmaf(0.05517166905792616f, f, 0.2426111221932161f);
   q = fmaf(q, f, 0.6932609854606553f);
   q = fmaf(q, f, 0.9999280735394012f);
-  const float r = __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
-  return y >= -126.f ? r : 0.f;
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 constexpr int FMA_EXP_EVERY = 4;        // every 4th column pair uses exp2_fma, the rest ex2.approx
 
