@@ -196,26 +196,6 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) {     // MN-major, S
   return smem_desc_sw128(saddr, VCH, 1024);
 }
 
-// 2^y on the FMA pipe, used for a share of the softmax exponentials so that the
-// MUFU unit (16 results per cycle per SM) is not the only source.  Cody-Waite
-// style range reduction y = n + f with n = round(y), f in [-1/2, 1/2] (the
-// 1.5 * 2^23 addend rounds y to an integer in the low mantissa bits), a cubic for
-// 2^f, and n added to the result's exponent field.  The cubic is the
-// relative-error minimax fit of 2^f on [-1/2, 1/2] found by a Remez exchange:
-// max relative error 7.5e-5 (also when evaluated in fp32), far below the bf16
-// rounding that P undergoes next.  y is clamped at -127 so that -inf (a masked
-// key) gives exactly 0.
-__device__ __forceinline__ float exp2_fma(float y) {
-  y = fmaxf(y, -127.f);
-  const float t = y + 12582912.f;
-  const float f = y - (t - 12582912.f);
-  float q = fmaf(0.05517166905792616f, f, 0.2426111221932161f);
-  q = fmaf(q, f, 0.6932609854606553f);
-  q = fmaf(q, f, 0.9999280735394012f);
-  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
-}
-constexpr int FMA_EXP_EVERY = 4;        // every 4th column pair uses exp2_fma, the rest ex2.approx
-
 // Word q (0..3) of a node's visibility mask, without dynamic register indexing.
 __device__ __forceinline__ uint32_t mask_word(const uint32_t (&w)[4], int q) {
   return q == 0 ? w[0] : (q == 1 ? w[1] : (q == 2 ? w[2] : w[3]));
@@ -305,10 +285,8 @@ __device__ __forceinline__ bool emit_p(const Ctx& cx, uint8_t* gbase, const floa
   uint32_t pk[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
-    const float y0 = fmaf(s[2 * c], scale_log2, -mb), y1 = fmaf(s[2 * c + 1], scale_log2, -mb);
-    const bool fma_pipe = (c % FMA_EXP_EVERY) == FMA_EXP_EVERY - 1;
-    const float p0 = fma_pipe ? exp2_fma(y0) : ex2(y0);
-    const float p1 = fma_pipe ? exp2_fma(y1) : ex2(y1);
+    const float p0 = ex2(fmaf(s[2 * c], scale_log2, -mb));
+    const float p1 = ex2(fmaf(s[2 * c + 1], scale_log2, -mb));
     rs[c & 3] += p0 + p1;
     pk[c] = pack_bf16x2(p0, p1);
   }
