@@ -96,9 +96,8 @@ enum Bar {
   S_FULL = K_EMPTY + NK,      // QK, both: S of the tile is in TMEM
   S_EMPTY = S_FULL + 1,       // QK leader: both CTAs copied S out (2 arrivals)
   P_FREE = S_EMPTY + 1,       // QK, both: the PV pair is done with a P slot
-  V_FULL = P_FREE + 2,        // PV, local: this CTA's V group landed
-  V_PEER = V_FULL + NVG,      // PV leader: the follower's V group landed (and tail cleared)
-  V_EMPTY = V_PEER + NVG,     // PV, both: the pair's MMAs are done with a V group
+  V_FULL = P_FREE + 2,        // PV leader: both CTAs' halves of a V group landed
+  V_EMPTY = V_FULL + NVG,     // PV, both: the pair's MMAs are done with a V group
   P_FULL = V_EMPTY + NVG,     // PV, local: this CTA's P slot arrived
   F_READY = P_FULL + 2,       // PV leader, per P slot: the follower's P slot arrived (and O rescaled)
   PV_TILE = F_READY + 2,      // PV, both: the pair's MMAs of a P tile are done
@@ -463,38 +462,48 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
 }
 
 // ====================================================================== PV pair roles
-// TMA producer (both PV CTAs): this CTA's 128 of every 256 latent columns of V.
+// TMA producer (both PV CTAs): this CTA's 128 of every 256 latent columns of V,
+// completing on the pair leader's barrier.
 __device__ __forceinline__ void pv_producer(const Ctx& cx, const CUtensorMap* tm_v, int64_t krow0,
                                             int ntiles) {
   bool ok = true;
   uint32_t gi = 0;
   const int col0 = (cx.rank & 1) * 128;
+  const bool leader = (cx.rank & 1) == 0;
+  const uint32_t lead = cx.rank & ~1u;
   for (int t = 0; t < 2 * ntiles && ok; ++t) {
     for (int kh = 0; kh < BN / VKEYS && ok; ++kh, ++gi) {
       const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN + kh * VKEYS);
       const uint32_t gs = gi % NVG, k = gi / NVG;
       if (!(ok = wait_bar(cx, cx.bar(V_EMPTY + gs), (k & 1u) ^ 1u))) break;
-      mbar_arrive_expect_tx(cx.bar(V_FULL + gs), VG);
+      if (leader) mbar_arrive_expect_tx(cx.bar(V_FULL + gs), 2 * VG);
       for (int hh = 0; hh < 2; ++hh)
         for (int a = 0; a < 2; ++a)
-          tma_load_2d(cx.base + V_OFF + gs * VG + (hh * 2 + a) * VCH, tm_v, hh * 256 + col0 + a * KC, krow,
-                      cx.bar(V_FULL + gs));
+          tma_load_2d_pair(cx.base + V_OFF + gs * VG + (hh * 2 + a) * VCH, tm_v, hh * 256 + col0 + a * KC,
+                           krow, cx.bar_of(lead, V_FULL + gs));
     }
   }
-  for (uint32_t j = (gi > NVG ? gi - NVG : 0); j < gi; ++j)
-    wait_bar(cx, cx.bar(V_FULL + j % NVG), (j / NVG) & 1u);
+  if (leader)
+    for (uint32_t j = (gi > NVG ? gi - NVG : 0); j < gi; ++j)
+      wait_bar(cx, cx.bar(V_FULL + j % NVG), (j / NVG) & 1u);
 }
 
 // Rows past the request's last key may hold anything (even NaN bit patterns); P
-// is 0 there but 0 * NaN is not, so clear them in this CTA's V group.
-__device__ __forceinline__ void clear_v_tail(uint8_t* gbase, uint32_t gs, int nv, int lane) {
+// is 0 there but 0 * NaN is not, so the pair leader clears them in both CTAs'
+// V group (the follower's through distributed shared memory) before its MMAs.
+// Only the last group of a key range can be partial.
+__device__ __forceinline__ void clear_v_tail(const Ctx& cx, uint8_t* gbase, uint32_t gs, int nv, int lane) {
   uint4* vg = reinterpret_cast<uint4*>(gbase + V_OFF + gs * VG);
+  const uint32_t peer_vg = map_to_rank(cx.base + V_OFF + gs * VG, cx.rank + 1);
   const int per_chunk = (VKEYS - nv) * 8;
   for (int idx = lane; idx < 4 * per_chunk; idx += 32) {
     const int q = idx / per_chunk, e = idx % per_chunk;
-    vg[q * (VCH / 16) + nv * 8 + e] = make_uint4(0u, 0u, 0u, 0u);
+    const int off = q * (VCH / 16) + nv * 8 + e;
+    vg[off] = make_uint4(0u, 0u, 0u, 0u);
+    st_cluster_v4(peer_vg + off * 16, 0u, 0u, 0u, 0u);
   }
   fence_proxy_async_cta();
+  fence_proxy_async_cluster();
   __syncwarp();
 }
 
@@ -545,13 +554,9 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, uint8_t* gbase, uint32_t t
     for (int kh = 0; kh < BN / VKEYS && ok; ++kh, ++gi) {
       const int nv = min(max(nvalid - kh * VKEYS, 0), VKEYS);
       const uint32_t gs = gi % NVG;
+      if (!leader) continue;                 // the leader waits for and consumes both halves
       if (!(ok = wait_warp(cx, cx.bar(V_FULL + gs), (gi / NVG) & 1u))) break;
-      if (nv < VKEYS) clear_v_tail(gbase, gs, nv, lane);
-      if (!leader) {
-        if (lane == 0) mbar_arrive_remote(cx.bar_of(lead, V_PEER + gs));
-        continue;
-      }
-      if (!(ok = wait_warp(cx, cx.bar(V_PEER + gs), (gi / NVG) & 1u, true))) break;
+      if (nv < VKEYS) clear_v_tail(cx, gbase, gs, nv, lane);
       tc_fence_after();
       if (lane == 0) {
         const uint32_t pa = cx.base + P_OFF + sb * PSLOT + kh * (BM * 128);
