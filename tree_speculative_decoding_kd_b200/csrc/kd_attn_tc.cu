@@ -69,11 +69,12 @@ constexpr int KC = 64;                  // columns per 128-byte swizzle atom
 constexpr int NCHUNK = 9;               // 8 latent chunks + 1 rope chunk
 constexpr int CHUNK = BN * KC * 2;      // 16 KB: 128 rows x 64 bf16 (also one K ring stage)
 constexpr int NQT = 8;                  // Q chunks held in TMEM (the rope chunk in shared memory)
-constexpr int NK = 8;                   // K ring stages
+constexpr int NK = 6;                   // K ring stages
 constexpr int VKEYS = 64;               // keys per V group
 constexpr int VCH = VKEYS * KC * 2;     // 8 KB: 64 keys x 64 latent columns
 constexpr int VG = 4 * VCH;             // this CTA's V group: 64 keys x (2 halves x 128 columns)
-constexpr int NVG = 4;                  // V ring depth
+constexpr int NVG = 3;                  // V ring depth
+constexpr int NP = 3;                   // P slots (staging in the QK CTA, landing in the PV CTA)
 constexpr int PBYTES = BM * BN * 2;     // one bf16 P tile (two 16 KB swizzle columns)
 constexpr int SLOT_ALPHA = PBYTES;      // f32 [128] per-row rescale factor
 constexpr int SLOT_FLAG = PBYTES + 512; // u32 rescale-needed flag
@@ -96,11 +97,11 @@ enum Bar {
   S_FULL = K_EMPTY + NK,      // QK, both: S of the tile is in TMEM
   S_EMPTY = S_FULL + 1,       // QK leader: both CTAs copied S out (2 arrivals)
   P_FREE = S_EMPTY + 1,       // QK, both: the PV pair is done with a P slot
-  V_FULL = P_FREE + 2,        // PV leader: both CTAs' halves of a V group landed
+  V_FULL = P_FREE + NP,       // PV leader: both CTAs' halves of a V group landed
   V_EMPTY = V_FULL + NVG,     // PV, both: the pair's MMAs are done with a V group
   P_FULL = V_EMPTY + NVG,     // PV, local: this CTA's P slot arrived
-  F_READY = P_FULL + 2,       // PV leader, per P slot: the follower's P slot arrived (and O rescaled)
-  PV_TILE = F_READY + 2,      // PV, both: the pair's MMAs of a P tile are done
+  F_READY = P_FULL + NP,      // PV leader, per P slot: the follower's P slot arrived (and O rescaled)
+  PV_TILE = F_READY + NP,     // PV, both: the pair's MMAs of a P tile are done
   O_DONE = PV_TILE + 1,       // PV, both: all MMAs of the unit are done
   EVENT = O_DONE + 1,         // PV, local: rescale request / end of loop
   CORR_DONE = EVENT + 1,      // PV, local: rescale applied (256 arrivals)
@@ -118,11 +119,11 @@ constexpr int OFF_XCH = 3072;           // f32 [2][128] max / sum exchange      
 static_assert(NBAR * 8 <= OFF_TMEM, "barrier block overflow");
 
 constexpr int Q_OFF = CTRL;                           // Q chunk 8 (rope)
-constexpr int STG_OFF = Q_OFF + CHUNK;                // P staging, 2 slots
-constexpr int K_OFF = STG_OFF + 2 * PSLOT;
+constexpr int STG_OFF = Q_OFF + CHUNK;                // P staging, NP slots
+constexpr int K_OFF = STG_OFF + NP * PSLOT;
 constexpr int QK_END = K_OFF + NK * CHUNK;
 constexpr int P_OFF = CTRL;
-constexpr int V_OFF = P_OFF + 2 * PSLOT;
+constexpr int V_OFF = P_OFF + NP * PSLOT;
 constexpr int PV_END = V_OFF + NVG * VG;
 constexpr int SMEM_BYTES = (QK_END > PV_END ? QK_END : PV_END) + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -195,7 +196,9 @@ __device__ __forceinline__ bool wait_group(const Ctx& cx, uint32_t bar, uint32_t
 __host__ __device__ constexpr int q_stage_off(int c) {
   return c < 4 ? STG_OFF + c * CHUNK : K_OFF + (NK - 4 + (c - 4)) * CHUNK;
 }
-static_assert(4 * CHUNK <= 2 * PSLOT && NK >= 4, "Q landing zones");
+static_assert(4 * CHUNK <= NP * PSLOT && NK >= 4, "Q landing zones");
+// the epilogue stages a 128 x 512 bf16 tile over the (then idle) P slots and V ring
+static_assert(8 * CHUNK <= NP * PSLOT + NVG * VG, "output staging");
 
 __device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {      // K-major, SW128
   return smem_desc_sw128(saddr, 16, 1024);
@@ -289,7 +292,7 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, uint32_t tmem, int ntiles)
 __device__ __forceinline__ bool emit_p(const Ctx& cx, uint8_t* gbase, const float (&x)[64], int u,
                                        float mb, float alpha, bool rescale_row, int r, int g,
                                        uint32_t peer_p, uint32_t peer_pfull, float& l_part) {
-  const uint32_t sb = u & 1;
+  const uint32_t sb = u % NP;
   float rs[4] = {0.f, 0.f, 0.f, 0.f};
   uint32_t pk[32];
 #pragma unroll
@@ -299,8 +302,8 @@ __device__ __forceinline__ bool emit_p(const Ctx& cx, uint8_t* gbase, const floa
     pk[c] = pack_bf16x2(p0, p1);
   }
   l_part += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-  // staging slot sb (and the partner's P slot sb) is free once the PV MMAs of P tile u-2 completed
-  if (!wait_group(cx, cx.bar(P_FREE + sb), ((u >> 1) & 1) ^ 1)) return false;
+  // staging slot sb (and the partner's P slot sb) is free once the PV MMAs of P tile u-NP completed
+  if (!wait_group(cx, cx.bar(P_FREE + sb), ((u / NP) & 1) ^ 1)) return false;
   const uint32_t stg = cx.base + STG_OFF + sb * PSLOT;
   const uint32_t prow = stg + g * (BM * 128) + (uint32_t)r * 128u;
 #pragma unroll
@@ -456,8 +459,8 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
     // the last P_FREE arrivals come from the PV pair's MMA completion: wait for them
     const int np = 2 * ntiles;
     if (ok)
-      for (int u = (np > 2 ? np - 2 : 0); u < np; ++u)
-        wait_bar(cx, cx.bar(P_FREE + (u & 1)), (u >> 1) & 1);
+      for (int u = (np > NP ? np - NP : 0); u < np; ++u)
+        wait_bar(cx, cx.bar(P_FREE + u % NP), (u / NP) & 1);
   }
 }
 
@@ -538,14 +541,14 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, uint8_t* gbase, uint32_t t
   bool ok = true;
   uint32_t gi = 0, nres = 0;
   for (int t = 0; t < 2 * ntiles && ok; ++t) {       // P tiles of 128 keys
-    const uint32_t sb = t & 1;
+    const uint32_t sb = t % NP;
     if (lane == 0) mbar_arrive_expect_tx(cx.bar(P_FULL + sb), SLOT_COPY);
-    if (!(ok = wait_warp(cx, cx.bar(P_FULL + sb), (t >> 1) & 1, true))) break;
+    if (!(ok = wait_warp(cx, cx.bar(P_FULL + sb), (t / NP) & 1, true))) break;
     if (!(ok = maybe_rescale(cx, gbase, t, sb, nres))) break;
     if (!leader) {
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(cx.bar_of(lead, F_READY + sb));
-    } else if (!(ok = wait_warp(cx, cx.bar(F_READY + sb), (t >> 1) & 1, true))) {
+    } else if (!(ok = wait_warp(cx, cx.bar(F_READY + sb), (t / NP) & 1, true))) {
       break;
     }
     tc_fence_after();
@@ -633,7 +636,7 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, cons
   const int64_t grow = (int64_t)b * rows_req + R;
   const int64_t prow = ((int64_t)sp * p.B * rows_req) + grow;
   if (p.splits == 1) {
-    // bf16 tile -> eight 128-row x 64-column boxes in the (now idle) V ring, laid out
+    // bf16 tile -> eight 128-row x 64-column boxes over the (now idle) P slots, laid out
     // with the 128-byte swizzle, then TMA stores; the per-request 3-D tensor map
     // clips rows past the request's last node.
     for (int c = 0; c < 256 / 64; ++c) {
@@ -645,7 +648,7 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, cons
 #pragma unroll
         for (int k = 0; k < 64; ++k) v[k] = 0u;
       }
-      const uint32_t box = cx.base + V_OFF + (g * 4 + c) * CHUNK + (uint32_t)r * 128u;
+      const uint32_t box = cx.base + P_OFF + (g * 4 + c) * CHUNK + (uint32_t)r * 128u;
 #pragma unroll
       for (int q = 0; q < 8; ++q)
         st_shared_v4(box + ((q ^ (r & 7)) << 4),
@@ -657,7 +660,7 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, cons
     fence_proxy_async_cta();
     named_bar_sync(1, GROUP);
     if (threadIdx.x == 64 && ok && mt < p.mtiles) {
-      for (int bx = 0; bx < 8; ++bx) tma_store_3d(tm_o, cx.base + V_OFF + bx * CHUNK, bx * KC, mt * BM, b);
+      for (int bx = 0; bx < 8; ++bx) tma_store_3d(tm_o, cx.base + P_OFF + bx * CHUNK, bx * KC, mt * BM, b);
       bulk_commit_group();
       bulk_wait_group_read0();
     }
