@@ -11,34 +11,32 @@
 // Because the latent is shared by all heads, a request's n*H query rows against
 // its keys form a dense (n*H x 576) . (576 x keys) contraction followed by a
 // (n*H x keys) . (keys x 512) one.  Rows are node-major (row = i*H + h) and cut
-// into 128-row M tiles; keys are streamed in 256-key tiles.
+// into 128-row M tiles; keys are streamed in 128-key tiles.
 //
 // The fp32 output accumulator of one M tile (128 x 512) fills all 512 TMEM
-// columns of an SM, leaving none for scores, so scores and outputs live on
-// different SMs.  A unit of work is two M tiles of one request and one key range,
-// run by a cluster of four CTAs:
-//   ranks 0, 1 ("QK" pair): S = Q K^T with 2-SM MMAs (cta_group::2, M = 256 =
-//       the two M tiles, N = 256 keys, K = 16), issued by rank 0.  Each CTA loads
-//       only its half (128 keys) of every K chunk into an 8-stage ring of 16 KB
-//       TMA boxes (128-byte swizzle); the pair's MMA reads both halves.  Each CTA
-//       keeps its M tile's eight 64-wide latent Q chunks in TMEM as the MMA's A
-//       operand (the rope chunk in shared memory) next to its 128 x 256 fp32 S.
-//       Two 4-warp softmax groups per CTA copy S into registers (freeing TMEM at
-//       once), keep an online max with a lazy rescale threshold, and emit bf16 P
-//       in 128-key halves: written into a local staging slot in the K-major
-//       swizzled layout the MMA reads, then moved to the partner PV CTA (rank + 2)
-//       by one bulk copy that completes on the partner's barrier.
-//   ranks 2, 3 ("PV" pair): O (128 x 512 fp32, its M tile) in each CTA's TMEM;
-//       O += P V with 2-SM MMAs (M = 256, N = 256 latent columns, K = 16 keys)
-//       issued by rank 2.  Each CTA loads only its 128 of every 256 latent
-//       columns of V (two 64-column MN-major boxes per 64-key group) into a
-//       4-deep ring.  Two 4-warp groups per CTA apply the rare O rescale and
-//       write the normalised output (or a split-KV partial).
-// Per SM this halves the K / V bytes loaded and read by the tensor cores, which
-// is what bounds a single-SM design.  No TMA multicast is used anywhere.
+// columns of an SM, leaving none for scores, so each unit of work runs on a
+// 2-CTA cluster with split roles:
+//   rank 0 ("QK" CTA): S = Q K^T for 256 keys at a time (M=128, N=256 MMAs, the
+//       shape that keeps the tensor pipe saturated from one issuing thread) into
+//       256 TMEM columns.  The eight 64-wide latent chunks of Q sit in the other 256
+//       TMEM columns and feed the MMA as its A operand from tensor memory; the rope
+//       chunk sits in shared memory.  Shared memory holds a 4-stage ring of
+//       256-key x 64-column K chunks (TMA, 128-byte swizzle) and two P staging
+//       slots.  Two 4-warp softmax groups copy S into registers (freeing TMEM for
+//       the next tile at once), keep an online max with a lazy rescale threshold,
+//       and emit P as two 128-key halves: each is written into a local staging slot
+//       in the K-major swizzled layout the MMA reads and moved to rank 1 by one
+//       thread with a single bulk copy that completes on rank 1's barrier.
+//   rank 1 ("PV" CTA): O (128 x 512 fp32) in TMEM; V as 64-key x 256-column
+//       groups (four 64-column MN-major boxes) in a 4-deep ring; O += P V as
+//       M=128, N=256, K=16 MMAs; two 4-warp groups apply the rare O rescale and
+//       write the normalised output (or a split-KV partial), 256 columns each.
+// QK work (576-deep) and PV work (512-deep) are nearly equal, so the pair keeps
+// both tensor pipes busy.  Both CTAs read the same c_kv tile (the second read
+// hits L2).  No TMA multicast is used anywhere.
 //
 // Every mbarrier wait is bounded (globaltimer); a wait that gives up raises
-// KD_DEV_TIMEOUT, marks the cluster aborted, and every role falls through to the
+// KD_DEV_TIMEOUT, marks both CTAs aborted, and every role falls through to the
 // common teardown (cluster barrier, TMEM release).
 
 #include <cuda.h>
@@ -58,54 +56,49 @@ namespace tc {
 
 using namespace ptx;
 
-constexpr int CLUSTER = 4;              // QK pair (ranks 0, 1) + PV pair (ranks 2, 3)
 constexpr int NTHREADS = 320;           // warp 0 TMA, warp 1 MMA, warps 2..9 two 4-warp groups
 constexpr int GROUP = 256;              // threads of the two 4-warp groups
-constexpr int BM = 128;                 // query rows per M tile (per CTA)
-constexpr int BQ = 256;                 // keys per QK tile (S = 128 x 256 per CTA)
-constexpr int KH = 128;                 // keys of a QK tile each QK CTA loads
+constexpr int BM = 128;                 // query rows per M tile
+constexpr int BQ = 256;                 // keys per QK tile (S = 128 x 256)
 constexpr int BN = 128;                 // keys per P / PV tile (two per QK tile)
 constexpr int KC = 64;                  // columns per 128-byte swizzle atom
 constexpr int NCHUNK = 9;               // 8 latent chunks + 1 rope chunk
-constexpr int CHUNK = BN * KC * 2;      // 16 KB: 128 rows x 64 bf16 (also one K ring stage)
+constexpr int CHUNK = BN * KC * 2;      // 16 KB: 128 rows x 64 bf16
+constexpr int KCHUNK = BQ * KC * 2;     // 32 KB: 256 keys x 64 bf16 (one K ring stage)
 constexpr int NQT = 8;                  // Q chunks held in TMEM (the rope chunk in shared memory)
-constexpr int NK = 6;                   // K ring stages
+constexpr int NK = 4;                   // K ring stages
 constexpr int VKEYS = 64;               // keys per V group
 constexpr int VCH = VKEYS * KC * 2;     // 8 KB: 64 keys x 64 latent columns
-constexpr int VG = 4 * VCH;             // this CTA's V group: 64 keys x (2 halves x 128 columns)
-constexpr int NVG = 3;                  // V ring depth
-constexpr int NP = 3;                   // P slots (staging in the QK CTA, landing in the PV CTA)
+constexpr int VG = 4 * VCH;             // one V group: 64 keys x 256 latent columns
+constexpr int NVG = 4;                  // V ring depth
 constexpr int PBYTES = BM * BN * 2;     // one bf16 P tile (two 16 KB swizzle columns)
 constexpr int SLOT_ALPHA = PBYTES;      // f32 [128] per-row rescale factor
-constexpr int SLOT_FLAG = PBYTES + 512; // u32 rescale-needed flag
-constexpr int SLOT_COPY = PBYTES + 528; // bytes moved to the PV CTA per P tile
+constexpr int SLOT_COPY = PBYTES + 512; // bytes that reach the PV CTA per P tile
+constexpr int WARP_ROWS_BYTES = 32 * 128;  // one warp's 32 rows of one 64-key swizzle atom
 constexpr int PSLOT = PBYTES + 1024;    // slot stride (keeps 1024-byte alignment)
 
-// TMEM columns of a QK CTA
-constexpr uint32_t TS = 0;              // S: 256 columns (128 x 256)
+// TMEM columns of the QK CTA
+constexpr uint32_t TS = 0;              // S: 256 columns (one 128 x 256 tile)
 constexpr uint32_t TQ = 256;            // Q chunks 0..7: 8 x 32 columns
 
-// control block (same offsets in every CTA so peers can address it)
+// control block (same offsets in both CTAs so the peer can address it)
 constexpr int CTRL = 4096;
 enum Bar {
-  Q_LAT = 0,                  // QK, local: this CTA's latent Q chunks landed
-  Q_ROPE = Q_LAT + 1,         // QK leader: both CTAs' rope Q chunks landed
-  QT_LOCAL = Q_ROPE + 1,      // QK, local: this CTA's Q is in TMEM (ring stages reusable)
-  QT_FULL = QT_LOCAL + 1,     // QK leader: both CTAs' Q in TMEM (2 arrivals)
-  K_FULL = QT_FULL + 1,       // QK leader: both halves of a K chunk landed
-  K_EMPTY = K_FULL + NK,      // QK, both: the pair's MMAs are done with a stage
-  S_FULL = K_EMPTY + NK,      // QK, both: S of the tile is in TMEM
-  S_EMPTY = S_FULL + 1,       // QK leader: both CTAs copied S out (2 arrivals)
-  P_FREE = S_EMPTY + 1,       // QK, both: the PV pair is done with a P slot
-  V_FULL = P_FREE + NP,       // PV leader: both CTAs' halves of a V group landed
-  V_EMPTY = V_FULL + NVG,     // PV, both: the pair's MMAs are done with a V group
-  P_FULL = V_EMPTY + NVG,     // PV, local: this CTA's P slot arrived
-  F_READY = P_FULL + NP,      // PV leader, per P slot: the follower's P slot arrived (and O rescaled)
-  PV_TILE = F_READY + NP,     // PV, both: the pair's MMAs of a P tile are done
-  O_DONE = PV_TILE + 1,       // PV, both: all MMAs of the unit are done
-  EVENT = O_DONE + 1,         // PV, local: rescale request / end of loop
-  CORR_DONE = EVENT + 1,      // PV, local: rescale applied (256 arrivals)
-  STATS = CORR_DONE + 1,      // PV, local: final row statistics arrived
+  Q_FULL = 0,
+  QT_FULL = Q_FULL + 1,
+  K_FULL = QT_FULL + 1,
+  K_EMPTY = K_FULL + NK,
+  S_FULL = K_EMPTY + NK,
+  S_EMPTY = S_FULL + 1,
+  P_FREE = S_EMPTY + 1,
+  V_FULL = P_FREE + 2,
+  V_EMPTY = V_FULL + NVG,
+  P_FULL = V_EMPTY + NVG,
+  PV_TILE = P_FULL + 2,
+  O_DONE = PV_TILE + 1,
+  EVENT = O_DONE + 1,
+  CORR_DONE = EVENT + 1,
+  STATS = CORR_DONE + 1,
   DRAIN = STATS + 1,
   NBAR = DRAIN + 1
 };
@@ -119,19 +112,19 @@ constexpr int OFF_XCH = 3072;           // f32 [2][128] max / sum exchange      
 static_assert(NBAR * 8 <= OFF_TMEM, "barrier block overflow");
 
 constexpr int Q_OFF = CTRL;                           // Q chunk 8 (rope)
-constexpr int STG_OFF = Q_OFF + CHUNK;                // P staging, NP slots
-constexpr int K_OFF = STG_OFF + NP * PSLOT;
-constexpr int QK_END = K_OFF + NK * CHUNK;
+constexpr int STG_OFF = Q_OFF + (NCHUNK - NQT) * CHUNK; // P staging, 2 slots
+constexpr int K_OFF = STG_OFF + 2 * PSLOT;
+constexpr int QK_END = K_OFF + NK * KCHUNK;
 constexpr int P_OFF = CTRL;
-constexpr int V_OFF = P_OFF + NP * PSLOT;
+constexpr int V_OFF = P_OFF + 2 * PSLOT;
 constexpr int PV_END = V_OFF + NVG * VG;
 constexpr int SMEM_BYTES = (QK_END > PV_END ? QK_END : PV_END) + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-constexpr uint32_t IDESC_QK = idesc_bf16(2 * BM, BQ, 0, 0);    // pair: Q, K both K-major
-constexpr uint32_t IDESC_PV = idesc_bf16(2 * BM, 256, 0, 1);   // pair: P K-major, V MN-major
-constexpr float RESCALE_THRESHOLD = 8.0f;                      // log2 units: P <= 2^8
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;              // 2 s per wait
+constexpr uint32_t IDESC_QK = idesc_bf16(BM, BQ, 0, 0);    // Q, K both K-major
+constexpr uint32_t IDESC_PV = idesc_bf16(BM, 256, 0, 1);   // P K-major, V MN-major
+constexpr float RESCALE_THRESHOLD = 8.0f;                  // log2 units: P <= 2^8
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;          // 2 s per wait
 
 struct Params {
   const int32_t* cache_lens;
@@ -143,22 +136,21 @@ struct Params {
   float* part_lse;
   int32_t* err;
   int64_t cap;
-  int B, n, H, W, mtiles, mpairs, splits;
+  int B, n, H, W, mtiles, splits;
   float scale_log2;
 };
 
 struct Ctx {
   uint32_t base;          // shared address of the aligned block
   volatile uint32_t* abort_flag;
-  uint32_t rank;          // cluster rank 0..3
+  uint32_t peer;          // cluster rank of the other CTA
   int32_t* err;
   __device__ uint32_t bar(int i) const { return base + 8u * (uint32_t)i; }
-  // barrier i of cluster rank r
-  __device__ uint32_t bar_of(uint32_t r, int i) const { return map_to_rank(bar(i), r); }
 };
 
-__device__ __noinline__ void abort_cluster(Ctx cx) {
-  for (uint32_t r = 0; r < CLUSTER; ++r) st_cluster_u32(map_to_rank(cx.base + OFF_ABORT, r), 1u);
+__device__ __noinline__ void abort_pair(Ctx cx) {
+  *cx.abort_flag = 1u;
+  st_cluster_u32(map_to_rank(cx.base + OFF_ABORT, cx.peer), 1u);
   raise_dev_error(cx.err, KD_DEV_TIMEOUT);
 }
 
@@ -173,7 +165,7 @@ __device__ __forceinline__ bool wait_bar(const Ctx& cx, uint32_t bar, uint32_t p
       if (*cx.abort_flag) return false;
       const uint64_t t = globaltimer();
       if (t0 == 0) t0 = t;
-      else if (t - t0 > WAIT_LIMIT_NS) { abort_cluster(cx); return false; }
+      else if (t - t0 > WAIT_LIMIT_NS) { abort_pair(cx); return false; }
     }
   }
 }
@@ -191,14 +183,11 @@ __device__ __forceinline__ bool wait_group(const Ctx& cx, uint32_t bar, uint32_t
   return !named_bar_red_or(1, GROUP, !ok);
 }
 
-// Shared-memory offset where TMA drops this CTA's Q latent chunk c (0..7) at the
-// start of a unit: the P staging area and the last four K ring stages are idle then.
+// Shared-memory offset where TMA drops Q latent chunk c (0..7) at the start of a unit.
 __host__ __device__ constexpr int q_stage_off(int c) {
-  return c < 4 ? STG_OFF + c * CHUNK : K_OFF + (NK - 4 + (c - 4)) * CHUNK;
+  return c < 4 ? STG_OFF + c * CHUNK : K_OFF + 2 * KCHUNK + (c - 4) * CHUNK;
 }
-static_assert(4 * CHUNK <= NP * PSLOT && NK >= 4, "Q landing zones");
-// the epilogue stages a 128 x 512 bf16 tile over the (then idle) P slots and V ring
-static_assert(8 * CHUNK <= NP * PSLOT + NVG * VG, "output staging");
+static_assert(4 * CHUNK <= 2 * PSLOT && 2 * KCHUNK + 4 * CHUNK <= NK * KCHUNK, "Q landing zones");
 
 __device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {      // K-major, SW128
   return smem_desc_sw128(saddr, 16, 1024);
@@ -206,6 +195,26 @@ __device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {      // K-major, SW
 __device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) {     // MN-major, SW128, 8 KB atoms
   return smem_desc_sw128(saddr, VCH, 1024);
 }
+
+// 2^y on the FMA pipe, used for a share of the softmax exponentials so that the
+// MUFU unit (16 results per cycle per SM) is not the only source.  Cody-Waite
+// style range reduction y = n + f with n = round(y), f in [-1/2, 1/2] (the
+// 1.5 * 2^23 addend rounds y to an integer in the low mantissa bits), a cubic for
+// 2^f, and n added to the result's exponent field.  The cubic is the
+// relative-error minimax fit of 2^f on [-1/2, 1/2] found by a Remez exchange:
+// max relative error 7.5e-5 (also when evaluated in fp32), far below the bf16
+// rounding that P undergoes next.  y is clamped at -127 so that -inf (a masked
+// key) gives exactly 0.
+__device__ __forceinline__ float exp2_fma(float y) {
+  y = fmaxf(y, -127.f);
+  const float t = y + 12582912.f;
+  const float f = y - (t - 12582912.f);
+  float q = fmaf(0.05517166905792616f, f, 0.2426111221932161f);
+  q = fmaf(q, f, 0.6932609854606553f);
+  q = fmaf(q, f, 0.9999280735394012f);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
+constexpr int FMA_EXP_EVERY = 4;        // every 4th column pair uses exp2_fma, the rest ex2.approx
 
 // Word q (0..3) of a node's visibility mask, without dynamic register indexing.
 __device__ __forceinline__ uint32_t mask_word(const uint32_t (&w)[4], int q) {
@@ -216,113 +225,115 @@ __device__ __forceinline__ float max4(float a, float b, float c, float d) {
   return fmaxf(fmaxf(a, b), fmaxf(c, d));
 }
 
-// ====================================================================== QK pair roles
-// TMA producer (both QK CTAs): this CTA's Q, then its 128-key half of every K chunk.
+// ====================================================================== QK CTA roles
+// TMA producer: Q chunks 7 and 8 once, then the K ring.
 __device__ __forceinline__ void qk_producer(const Ctx& cx, const CUtensorMap* tm_qa,
                                             const CUtensorMap* tm_qr, const CUtensorMap* tm_c,
                                             const CUtensorMap* tm_r, int qrow0, int64_t krow0,
-                                            int ntiles, bool leader) {
+                                            int ntiles) {
   const uint32_t base = cx.base;
-  const uint32_t lead = cx.rank & ~1u;
-  mbar_arrive_expect_tx(cx.bar(Q_LAT), NQT * CHUNK);
-  for (int c = 0; c < NQT; ++c) tma_load_2d(base + q_stage_off(c), tm_qa, c * KC, qrow0, cx.bar(Q_LAT));
-  if (leader) mbar_arrive_expect_tx(cx.bar(Q_ROPE), 2 * CHUNK);
-  tma_load_2d_pair(base + Q_OFF, tm_qr, 0, qrow0, cx.bar_of(lead, Q_ROPE));
+  // Q: latent chunks 0..3 land in the (still unused) P staging area, chunks 4..7 in
+  // K ring stages 2..3; the softmax groups move them into TMEM.  The rope chunk stays.
+  mbar_arrive_expect_tx(cx.bar(Q_FULL), NCHUNK * CHUNK);
+  for (int c = 0; c < NQT; ++c) tma_load_2d(base + q_stage_off(c), tm_qa, c * KC, qrow0, cx.bar(Q_FULL));
+  tma_load_2d(base + Q_OFF, tm_qr, 0, qrow0, cx.bar(Q_FULL));
   uint32_t it = 0;
   bool ok = true;
   for (int t = 0; t < ntiles && ok; ++t) {
-    const int32_t krow = (int32_t)(krow0 + (int64_t)t * BQ + (cx.rank & 1) * KH);
+    const int32_t krow = (int32_t)(krow0 + (int64_t)t * BQ);
     for (int c = 0; c < NCHUNK; ++c, ++it) {
       const uint32_t st = it % NK, k = it / NK;
       if (!(ok = wait_bar(cx, cx.bar(K_EMPTY + st), (k & 1u) ^ 1u))) break;
-      // the last four stages held this CTA's Q until it moved to TMEM
-      if (it == NK - 4 && !(ok = wait_bar(cx, cx.bar(QT_LOCAL), 0))) break;
-      if (leader) mbar_arrive_expect_tx(cx.bar(K_FULL + st), 2 * CHUNK);
-      if (c < 8) tma_load_2d_pair(base + K_OFF + st * CHUNK, tm_c, c * KC, krow, cx.bar_of(lead, K_FULL + st));
-      else tma_load_2d_pair(base + K_OFF + st * CHUNK, tm_r, 0, krow, cx.bar_of(lead, K_FULL + st));
+      if (it == 2 && !(ok = wait_bar(cx, cx.bar(QT_FULL), 0))) break;   // stages 2, 3 held Q
+      mbar_arrive_expect_tx(cx.bar(K_FULL + st), KCHUNK);
+      if (c < 8) tma_load_2d(base + K_OFF + st * KCHUNK, tm_c, c * KC, krow, cx.bar(K_FULL + st));
+      else tma_load_2d(base + K_OFF + st * KCHUNK, tm_r, 0, krow, cx.bar(K_FULL + st));
     }
   }
-  // every armed stage must have landed before the CTA may exit (the leader sees
-  // both halves complete; the follower waits for the leader's matching drain via
-  // the final cluster barrier)
-  wait_bar(cx, cx.bar(Q_LAT), 0);
-  if (leader) {
-    wait_bar(cx, cx.bar(Q_ROPE), 0);
-    for (uint32_t j = (it > NK ? it - NK : 0); j < it; ++j)
-      wait_bar(cx, cx.bar(K_FULL + j % NK), (j / NK) & 1u);
-  }
+  // every armed stage must have landed before the CTA may exit
+  wait_bar(cx, cx.bar(Q_FULL), 0);
+  for (uint32_t j = (it > NK ? it - NK : 0); j < it; ++j)
+    wait_bar(cx, cx.bar(K_FULL + j % NK), (j / NK) & 1u);
 }
 
-// MMA issuer (QK leader only): S = Q K^T for both M tiles with 2-SM MMAs.
+// MMA issuer: S[t % 2] = Q K^T (A from TMEM for chunks 0..7, from shared memory for 8).
 __device__ __forceinline__ void qk_mma(const Ctx& cx, uint32_t tmem, int ntiles) {
   const uint32_t base = cx.base;
-  bool ok = wait_bar(cx, cx.bar(Q_ROPE), 0) && wait_bar(cx, cx.bar(QT_FULL), 0, true);
+  bool ok = wait_bar(cx, cx.bar(Q_FULL), 0) && wait_bar(cx, cx.bar(QT_FULL), 0);
   tc_fence_after();
   uint32_t it = 0;
   for (int t = 0; t < ntiles && ok; ++t) {
-    if (!(ok = wait_bar(cx, cx.bar(S_EMPTY), (t & 1) ^ 1, true))) break;
+    if (!(ok = wait_bar(cx, cx.bar(S_EMPTY), (t & 1) ^ 1))) break;
     tc_fence_after();
     const uint32_t d = tmem + TS;
     for (int c = 0; c < NCHUNK; ++c, ++it) {
       const uint32_t st = it % NK;
       if (!(ok = wait_bar(cx, cx.bar(K_FULL + st), (it / NK) & 1u))) break;
       tc_fence_after();
-      const uint32_t b0 = base + K_OFF + st * CHUNK;
+      const uint32_t b0 = base + K_OFF + st * KCHUNK;
       if (c < NQT) {
 #pragma unroll
         for (int kk = 0; kk < KC / 16; ++kk)
-          mma2_bf16_ts(d, tmem + TQ + c * 32 + kk * 8, desc_k(b0 + kk * 32), IDESC_QK, (c | kk) != 0);
+          mma_bf16_ts(d, tmem + TQ + c * 32 + kk * 8, desc_k(b0 + kk * 32), IDESC_QK, (c | kk) != 0);
       } else {
+        const uint32_t a0 = base + Q_OFF + (c - NQT) * CHUNK;
 #pragma unroll
         for (int kk = 0; kk < KC / 16; ++kk)
-          mma2_bf16_ss(d, desc_k(base + Q_OFF + kk * 32), desc_k(b0 + kk * 32), IDESC_QK, 1u);
+          mma_bf16_ss(d, desc_k(a0 + kk * 32), desc_k(b0 + kk * 32), IDESC_QK, 1u);
       }
-      tc_commit_pair_mc(cx.bar(K_EMPTY + st), 0x3);
+      tc_commit(cx.bar(K_EMPTY + st));
     }
-    if (ok) tc_commit_pair_mc(cx.bar(S_FULL), 0x3);
+    if (ok) tc_commit(cx.bar(S_FULL));
   }
-  tc_commit_pair_mc(cx.bar(DRAIN), 0x3);
+  tc_commit(cx.bar(DRAIN));
   wait_bar(cx, cx.bar(DRAIN), 0);
 }
 
-// One 128-key half of a QK tile: exponentiate this thread's 64 columns against
-// the row reference mb, add them to the running sum, and ship the bf16 P tile
-// (plus the per-row rescale factor for the PV side) through staging slot u % 2
-// to the partner PV CTA.
-__device__ __forceinline__ bool emit_p(const Ctx& cx, uint8_t* gbase, const float (&x)[64], int u,
-                                       float mb, float alpha, bool rescale_row, int r, int g,
-                                       uint32_t peer_p, uint32_t peer_pfull, float& l_part) {
-  const uint32_t sb = u % NP;
+// One 128-key half of a QK tile.  Each softmax warp works alone here: it
+// exponentiates its 32 rows x 64 columns (raw scores s, p = 2^(s * scale_log2 - m)),
+// adds them to the rows' running sums, writes them into its own contiguous 4 KB
+// slice of staging slot u % 2 (32 rows of one 64-key atom of the K-major,
+// 128-byte-swizzled P layout) and ships that slice with one bulk copy that
+// completes on the PV CTA's barrier.  Group 0 warps also ship the rows' rescale
+// factors.
+__device__ __forceinline__ bool emit_p(const Ctx& cx, uint8_t* gbase, const float (&s)[64], int u,
+                                       float scale_log2, float mb, float alpha, int r, int g,
+                                       int quad, uint32_t peer_p, uint32_t peer_ctrl, float& l_part) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t sb = u & 1;
   float rs[4] = {0.f, 0.f, 0.f, 0.f};
   uint32_t pk[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
-    const float p0 = ex2(x[2 * c] - mb), p1 = ex2(x[2 * c + 1] - mb);
+    const float y0 = fmaf(s[2 * c], scale_log2, -mb), y1 = fmaf(s[2 * c + 1], scale_log2, -mb);
+    const bool fma_pipe = (c % FMA_EXP_EVERY) == FMA_EXP_EVERY - 1;
+    const float p0 = fma_pipe ? exp2_fma(y0) : ex2(y0);
+    const float p1 = fma_pipe ? exp2_fma(y1) : ex2(y1);
     rs[c & 3] += p0 + p1;
     pk[c] = pack_bf16x2(p0, p1);
   }
   l_part += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-  // staging slot sb (and the partner's P slot sb) is free once the PV MMAs of P tile u-NP completed
-  if (!wait_group(cx, cx.bar(P_FREE + sb), ((u / NP) & 1) ^ 1)) return false;
+  // staging slot sb (and the peer's P slot sb) is free once the PV MMAs of P tile u-2 completed
+  if (!wait_warp(cx, cx.bar(P_FREE + sb), ((u >> 1) & 1) ^ 1)) return false;
+  const uint32_t slice = (uint32_t)(g * (BM * 128) + quad * WARP_ROWS_BYTES);
   const uint32_t stg = cx.base + STG_OFF + sb * PSLOT;
-  const uint32_t prow = stg + g * (BM * 128) + (uint32_t)r * 128u;
+  const uint32_t prow = stg + slice + (uint32_t)lane * 128u;
 #pragma unroll
   for (int q = 0; q < 8; ++q)
     st_shared_v4(prow + ((q ^ (r & 7)) << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-  float* stgf = reinterpret_cast<float*>(gbase + STG_OFF + sb * PSLOT);
-  if (g == 0) stgf[(SLOT_ALPHA >> 2) + r] = alpha;
+  if (g == 0) reinterpret_cast<float*>(gbase + STG_OFF + sb * PSLOT + SLOT_ALPHA)[r] = alpha;
   fence_proxy_async_cta();
-  const bool any = named_bar_red_or(1, GROUP, rescale_row);
-  if (threadIdx.x == 64) {
-    reinterpret_cast<uint32_t*>(stgf)[SLOT_FLAG >> 2] = any ? 1u : 0u;
-    fence_proxy_async_cta();
-    bulk_copy_to_peer(peer_p + sb * PSLOT, stg, SLOT_COPY, peer_pfull + 8u * sb);
+  __syncwarp();
+  if (lane == 0) {
+    const uint32_t dst = peer_p + sb * PSLOT, bar = peer_ctrl + 8u * P_FULL + 8u * sb;
+    bulk_copy_to_peer(dst + slice, stg + slice, WARP_ROWS_BYTES, bar);
+    if (g == 0)
+      bulk_copy_to_peer(dst + SLOT_ALPHA + quad * 128, stg + SLOT_ALPHA + quad * 128, 128, bar);
   }
   return true;
 }
 
-// Softmax groups (both QK CTAs): thread (g, r) owns row r of this CTA's M tile
-// and key columns [64 g, 64 g + 64) of each 128-key half of every tile.
+// Softmax groups: thread (g, r) owns row r and key columns [64 g, 64 g + 64) of every tile.
 __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8_t* gbase,
                                            uint32_t tmem, int b, int mt, int sp, int64_t L,
                                            int64_t kbeg, int ntiles) {
@@ -336,14 +347,12 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
   const bool valid = R < rows_req;
   const int node = valid ? R / H : 0;
   float* xch = reinterpret_cast<float*>(gbase + OFF_XCH);
-  const uint32_t lead = cx.rank & ~1u;
-  const uint32_t partner = cx.rank + 2;
 
   // ---- Q chunks 0..7 of this row into TMEM (group 0: chunks 0..3, group 1: 4..7),
   //      read back from the 128-byte-swizzled TMA landing zones
   {
     // an empty key partition issues no loads at all (its producer does not run)
-    const bool okq = ntiles > 0 && wait_group(cx, cx.bar(Q_LAT), 0);
+    const bool okq = ntiles > 0 && wait_group(cx, cx.bar(Q_FULL), 0);
     if (okq) {
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
@@ -360,11 +369,7 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
       tmem_wait_st();
     }
     tc_fence_before();
-    named_bar_sync(1, GROUP);
-    if (threadIdx.x == 64) {
-      mbar_arrive(cx.bar(QT_LOCAL));
-      mbar_arrive_remote(cx.bar_of(lead, QT_FULL));
-    }
+    mbar_arrive(cx.bar(QT_FULL));
   }
 
   const int W = p.W;
@@ -377,32 +382,34 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
     if (p.positions && p.positions[(size_t)b * n + node] != (int32_t)(L + depth))
       raise_dev_error(p.err, KD_DEV_BAD_POSITION);
   }
-  const uint32_t peer_p = map_to_rank(cx.base + P_OFF, partner);
-  const uint32_t peer_ctrl = map_to_rank(cx.base, partner);
-  const uint32_t peer_pfull = peer_ctrl + 8u * P_FULL;
-  float m_ref = -INFINITY, l_part = 0.f;
+  const uint32_t peer_p = map_to_rank(cx.base + P_OFF, cx.peer);
+  const uint32_t peer_ctrl = map_to_rank(cx.base, cx.peer);
+  const uint32_t pair_bar = 2 + quad;          // the two warps (one per group) that share rows
+  const float sl2 = p.scale_log2;
+  float m_ref = -INFINITY, l_part = 0.f;       // reference max in log2 units; partial row sum
   bool ok = true;
-  for (int t = 0; t < ntiles && ok; ++t) {
-    if (!(ok = wait_group(cx, cx.bar(S_FULL), t & 1))) break;
-    tc_fence_after();
-    // this thread's columns: keys 64 g .. 64 g + 63 of each 128-key half h of the tile
+  for (int t = 0; t < ntiles; ++t) {
+    // a warp whose wait gave up still meets its partner warp at the pair barrier
+    // below, so both leave the loop together
+    const bool okw = ok && wait_warp(cx, cx.bar(S_FULL), t & 1);
+    // this thread's columns: keys 64 g .. 64 g + 63 of each 128-key half h of the tile (raw scores)
     float x[2][64];
-    {
+    if (okw) {
+      tc_fence_after();
       uint32_t u0[64], u1[64];
       tmem_ld64(lane_addr + TS + g * 64, u0);
       tmem_ld64(lane_addr + TS + BN + g * 64, u1);
       tmem_wait_ld();
 #pragma unroll
       for (int k = 0; k < 64; ++k) {
-        x[0][k] = __uint_as_float(u0[k]) * p.scale_log2;
-        x[1][k] = __uint_as_float(u1[k]) * p.scale_log2;
+        x[0][k] = __uint_as_float(u0[k]);
+        x[1][k] = __uint_as_float(u1[k]);
       }
-    }
-    tc_fence_before();
-    named_bar_sync(1, GROUP);
-    if (threadIdx.x == 64) {                   // this CTA's S is out of TMEM
-      if (cx.rank == lead) mbar_arrive(cx.bar(S_EMPTY));
-      else mbar_arrive_remote(cx.bar_of(lead, S_EMPTY));
+      tc_fence_before();
+      mbar_arrive(cx.bar(S_EMPTY));            // TMEM free for the next tile's MMAs
+    } else {
+#pragma unroll
+      for (int k = 0; k < 64; ++k) x[0][k] = x[1][k] = -INFINITY;
     }
     // mask: only keys at or beyond L need it
 #pragma unroll
@@ -426,171 +433,145 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
         mx[0] = fmaxf(mx[0], x[h][c]); mx[1] = fmaxf(mx[1], x[h][c + 1]);
         mx[2] = fmaxf(mx[2], x[h][c + 2]); mx[3] = fmaxf(mx[3], x[h][c + 3]);
       }
-    xch[g * BM + r] = max4(mx[0], mx[1], mx[2], mx[3]);
-    named_bar_sync(1, GROUP);
+    // row max over both groups' columns: exchange with the partner warp only
+    xch[g * BM + r] = max4(mx[0], mx[1], mx[2], mx[3]) * sl2;
+    if (named_bar_red_or(pair_bar, 64, !okw)) {
+      ok = false;
+      break;
+    }
     const float tmax = fmaxf(xch[r], xch[BM + r]);
+    named_bar_sync(pair_bar, 64);              // both reads done before the next write
     float alpha = 1.f;
-    bool rescale_row = false;
     if (tmax > m_ref + RESCALE_THRESHOLD) {
-      if (m_ref != -INFINITY) {
-        alpha = ex2(m_ref - tmax);
-        rescale_row = true;
-      } else {
-        alpha = 0.f;
-      }
+      alpha = m_ref != -INFINITY ? ex2(m_ref - tmax) : 0.f;
       l_part *= alpha;
       m_ref = tmax;
     }
     const float mb = m_ref == -INFINITY ? 0.f : m_ref;
-    ok = emit_p(cx, gbase, x[0], 2 * t, mb, alpha, rescale_row, r, g, peer_p, peer_pfull, l_part) &&
-         emit_p(cx, gbase, x[1], 2 * t + 1, mb, 1.f, false, r, g, peer_p, peer_pfull, l_part);
+    ok = emit_p(cx, gbase, x[0], 2 * t, sl2, mb, alpha, r, g, quad, peer_p, peer_ctrl, l_part) &&
+         emit_p(cx, gbase, x[1], 2 * t + 1, sl2, mb, 1.f, r, g, quad, peer_p, peer_ctrl, l_part);
   }
   // final row statistics for the epilogue: l = both groups' partial sums
-  named_bar_sync(1, GROUP);
   xch[g * BM + r] = l_part;
-  named_bar_sync(1, GROUP);
+  ok = !named_bar_red_or(pair_bar, 64, !ok);
   if (g == 0) {
     st_cluster_u32(peer_ctrl + OFF_MFIN + r * 4, __float_as_uint(m_ref));
     st_cluster_u32(peer_ctrl + OFF_LFIN + r * 4, __float_as_uint(xch[r] + xch[BM + r]));
+    __syncwarp();
+    if (lane == 0) mbar_arrive_remote(peer_ctrl + 8u * STATS);
   }
-  named_bar_sync(1, GROUP);
+  ok = !named_bar_red_or(1, GROUP, !ok);
   if (threadIdx.x == 64) {
-    mbar_arrive_remote(peer_ctrl + 8u * STATS);
-    // the last P_FREE arrivals come from the PV pair's MMA completion: wait for them
+    // the last P_FREE arrivals come from the peer's MMA completion: wait for them
     const int np = 2 * ntiles;
     if (ok)
-      for (int u = (np > NP ? np - NP : 0); u < np; ++u)
-        wait_bar(cx, cx.bar(P_FREE + u % NP), (u / NP) & 1);
+      for (int u = (np > 2 ? np - 2 : 0); u < np; ++u)
+        wait_bar(cx, cx.bar(P_FREE + (u & 1)), (u >> 1) & 1);
   }
 }
 
-// ====================================================================== PV pair roles
-// TMA producer (both PV CTAs): this CTA's 128 of every 256 latent columns of V,
-// completing on the pair leader's barrier.
+// ====================================================================== PV CTA roles
 __device__ __forceinline__ void pv_producer(const Ctx& cx, const CUtensorMap* tm_v, int64_t krow0,
                                             int ntiles) {
   bool ok = true;
   uint32_t gi = 0;
-  const int col0 = (cx.rank & 1) * 128;
-  const bool leader = (cx.rank & 1) == 0;
-  const uint32_t lead = cx.rank & ~1u;
   for (int t = 0; t < 2 * ntiles && ok; ++t) {
-    for (int kh = 0; kh < BN / VKEYS && ok; ++kh, ++gi) {
+    for (int kh = 0; kh < BN / VKEYS && ok; ++kh) {
       const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN + kh * VKEYS);
-      const uint32_t gs = gi % NVG, k = gi / NVG;
-      if (!(ok = wait_bar(cx, cx.bar(V_EMPTY + gs), (k & 1u) ^ 1u))) break;
-      if (leader) mbar_arrive_expect_tx(cx.bar(V_FULL + gs), 2 * VG);
-      for (int hh = 0; hh < 2; ++hh)
-        for (int a = 0; a < 2; ++a)
-          tma_load_2d_pair(cx.base + V_OFF + gs * VG + (hh * 2 + a) * VCH, tm_v, hh * 256 + col0 + a * KC,
-                           krow, cx.bar_of(lead, V_FULL + gs));
+      for (int hh = 0; hh < 2; ++hh, ++gi) {
+        const uint32_t gs = gi % NVG, k = gi / NVG;
+        if (!(ok = wait_bar(cx, cx.bar(V_EMPTY + gs), (k & 1u) ^ 1u))) break;
+        mbar_arrive_expect_tx(cx.bar(V_FULL + gs), VG);
+        for (int q = 0; q < 4; ++q)
+          tma_load_2d(cx.base + V_OFF + gs * VG + q * VCH, tm_v, (hh * 4 + q) * KC, krow,
+                      cx.bar(V_FULL + gs));
+      }
     }
   }
-  if (leader)
-    for (uint32_t j = (gi > NVG ? gi - NVG : 0); j < gi; ++j)
-      wait_bar(cx, cx.bar(V_FULL + j % NVG), (j / NVG) & 1u);
+  for (uint32_t j = (gi > NVG ? gi - NVG : 0); j < gi; ++j)
+    wait_bar(cx, cx.bar(V_FULL + j % NVG), (j / NVG) & 1u);
 }
 
-// Rows past the request's last key may hold anything (even NaN bit patterns); P
-// is 0 there but 0 * NaN is not, so the pair leader clears them in both CTAs'
-// V group (the follower's through distributed shared memory) before its MMAs.
-// Only the last group of a key range can be partial.
-__device__ __forceinline__ void clear_v_tail(const Ctx& cx, uint8_t* gbase, uint32_t gs, int nv, int lane) {
-  uint4* vg = reinterpret_cast<uint4*>(gbase + V_OFF + gs * VG);
-  const uint32_t peer_vg = map_to_rank(cx.base + V_OFF + gs * VG, cx.rank + 1);
-  const int per_chunk = (VKEYS - nv) * 8;
-  for (int idx = lane; idx < 4 * per_chunk; idx += 32) {
-    const int q = idx / per_chunk, e = idx % per_chunk;
-    const int off = q * (VCH / 16) + nv * 8 + e;
-    vg[off] = make_uint4(0u, 0u, 0u, 0u);
-    st_cluster_v4(peer_vg + off * 16, 0u, 0u, 0u, 0u);
-  }
-  fence_proxy_async_cta();
-  fence_proxy_async_cluster();
-  __syncwarp();
-}
-
-// If this CTA's P slot asks for it, rescale O (after the pair's MMAs of the
-// previous P tile are done) through the local correction groups.
-__device__ __forceinline__ bool maybe_rescale(const Ctx& cx, uint8_t* gbase, int t, uint32_t sb,
-                                              uint32_t& nres) {
-  const int lane = threadIdx.x & 31;
-  volatile uint32_t* ctrl = reinterpret_cast<volatile uint32_t*>(gbase);
-  const uint32_t flag = *reinterpret_cast<volatile uint32_t*>(gbase + P_OFF + sb * PSLOT + SLOT_FLAG);
-  if (!(flag && t > 0)) return true;
-  if (!wait_warp(cx, cx.bar(PV_TILE), (t - 1) & 1)) return false;
-  if (lane == 0) {
-    ctrl[OFF_EVTYPE >> 2] = 1u;
-    ctrl[OFF_EVTILE >> 2] = sb;
-    mbar_arrive(cx.bar(EVENT));
-  }
-  if (!wait_warp(cx, cx.bar(CORR_DONE), nres & 1u)) return false;
-  ++nres;
-  return true;
-}
-
-// MMA warp of the PV pair.  The leader issues O += P V for both M tiles; the
-// follower forwards its readiness (P slot arrived and O rescaled, V group landed
-// and tail cleared) to the leader.
 __device__ __forceinline__ void pv_mma(const Ctx& cx, uint8_t* gbase, uint32_t tmem, int64_t kbeg,
                                        int64_t nkeys, int ntiles) {
   const int lane = threadIdx.x & 31;
-  const bool leader = (cx.rank & 1) == 0;
-  const uint32_t lead = cx.rank & ~1u;
   volatile uint32_t* ctrl = reinterpret_cast<volatile uint32_t*>(gbase);
   bool ok = true;
   uint32_t gi = 0, nres = 0;
-  for (int t = 0; t < 2 * ntiles && ok; ++t) {       // P tiles of 128 keys
-    const uint32_t sb = t % NP;
+  for (int t = 0; t < 2 * ntiles && ok; ++t) {      // P tiles of 128 keys
+    const uint32_t sb = t & 1;
     if (lane == 0) mbar_arrive_expect_tx(cx.bar(P_FULL + sb), SLOT_COPY);
-    if (!(ok = wait_warp(cx, cx.bar(P_FULL + sb), (t / NP) & 1, true))) break;
-    if (!(ok = maybe_rescale(cx, gbase, t, sb, nres))) break;
-    if (!leader) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(cx.bar_of(lead, F_READY + sb));
-    } else if (!(ok = wait_warp(cx, cx.bar(F_READY + sb), (t / NP) & 1, true))) {
-      break;
+    if (!(ok = wait_warp(cx, cx.bar(P_FULL + sb), (t >> 1) & 1, true))) break;
+    // rows whose reference max moved (alpha not 1; alpha 0 means the row had no
+    // visible key yet, so its O row is still 0) need O rescaled first
+    const volatile float* al = reinterpret_cast<const volatile float*>(gbase + P_OFF + sb * PSLOT + SLOT_ALPHA);
+    bool moved = false;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float a = al[lane * 4 + q];
+      moved |= (a != 1.f && a != 0.f);
+    }
+    const bool flag = __any_sync(0xffffffffu, moved);
+    if (flag && t > 0) {
+      // every earlier PV MMA must be done before O is rescaled
+      if (!(ok = wait_warp(cx, cx.bar(PV_TILE), (t - 1) & 1))) break;
+      if (lane == 0) {
+        ctrl[OFF_EVTYPE >> 2] = 1u;
+        ctrl[OFF_EVTILE >> 2] = sb;
+        mbar_arrive(cx.bar(EVENT));
+      }
+      if (!(ok = wait_warp(cx, cx.bar(CORR_DONE), nres & 1u))) break;
+      ++nres;
     }
     tc_fence_after();
     const int64_t kt = kbeg + (int64_t)t * BN;
     const int nvalid = (int)((nkeys - kt) < BN ? (nkeys - kt) : BN);
-    for (int kh = 0; kh < BN / VKEYS && ok; ++kh, ++gi) {
+    for (int kh = 0; kh < BN / VKEYS && ok; ++kh) {
       const int nv = min(max(nvalid - kh * VKEYS, 0), VKEYS);
-      const uint32_t gs = gi % NVG;
-      if (!leader) continue;                 // the leader waits for and consumes both halves
-      if (!(ok = wait_warp(cx, cx.bar(V_FULL + gs), (gi / NVG) & 1u))) break;
-      if (nv < VKEYS) clear_v_tail(cx, gbase, gs, nv, lane);
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t pa = cx.base + P_OFF + sb * PSLOT + kh * (BM * 128);
-        const uint32_t vb = cx.base + V_OFF + gs * VG;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
+      for (int hh = 0; hh < 2 && ok; ++hh, ++gi) {
+        const uint32_t gs = gi % NVG;
+        if (!(ok = wait_warp(cx, cx.bar(V_FULL + gs), (gi / NVG) & 1u))) break;
+        if (nv < VKEYS) {
+          // rows past the request's last key may hold anything (even NaN bit
+          // patterns); P is 0 there but 0 * NaN is not, so clear them
+          uint4* vg = reinterpret_cast<uint4*>(gbase + V_OFF + gs * VG);
+          const int per_chunk = (VKEYS - nv) * 8;
+          for (int idx = lane; idx < 4 * per_chunk; idx += 32) {
+            const int q = idx / per_chunk, e = idx % per_chunk;
+            vg[q * (VCH / 16) + nv * 8 + e] = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_cta();
+          __syncwarp();
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t pa = cx.base + P_OFF + sb * PSLOT + kh * (BM * 128);
+          const uint32_t vb = cx.base + V_OFF + gs * VG;
 #pragma unroll
           for (int ks = 0; ks < VKEYS / 16; ++ks)
-            mma2_bf16_ss(tmem + hh * 256, desc_k(pa + ks * 32), desc_mn(vb + hh * 2 * VCH + ks * 2048),
-                         IDESC_PV, (t > 0 || kh > 0 || ks > 0) ? 1u : 0u);
-        tc_commit_pair_mc(cx.bar(V_EMPTY + gs), 0xC);
+            mma_bf16_ss(tmem + hh * 256, desc_k(pa + ks * 32), desc_mn(vb + ks * 2048), IDESC_PV,
+                        (t > 0 || kh > 0 || ks > 0) ? 1u : 0u);
+          tc_commit(cx.bar(V_EMPTY + gs));
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
-    if (leader && ok && lane == 0) {
-      tc_commit_pair_mc(cx.bar(PV_TILE), 0xC);
-      tc_commit_pair_mc(cx.bar(P_FREE + sb), 0x3);
+    if (ok && lane == 0) {
+      tc_commit(cx.bar(PV_TILE));
+      tc_commit_mc(cx.bar(P_FREE + sb), (uint16_t)(1u << cx.peer));
     }
     __syncwarp();
   }
   if (lane == 0) {
-    if (leader && ntiles > 0) tc_commit_pair_mc(cx.bar(O_DONE), 0xC);
-    else if (ntiles == 0) mbar_arrive(cx.bar(O_DONE));
+    if (ntiles > 0) tc_commit(cx.bar(O_DONE));
+    else mbar_arrive(cx.bar(O_DONE));
     ctrl[OFF_EVTYPE >> 2] = 2u;
     mbar_arrive(cx.bar(EVENT));
   }
   __syncwarp();
 }
 
-// Correction / epilogue groups (both PV CTAs): thread (g, r) owns row r of this
-// CTA's M tile and O columns [256 g, 256 g + 256).
+// Correction / epilogue groups: thread (g, r) owns row r, O columns [256 g, 256 g + 256).
 __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, const CUtensorMap* tm_o,
                                             uint8_t* gbase, uint32_t tmem, int b, int mt, int sp,
                                             int ntiles) {
@@ -636,7 +617,7 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, cons
   const int64_t grow = (int64_t)b * rows_req + R;
   const int64_t prow = ((int64_t)sp * p.B * rows_req) + grow;
   if (p.splits == 1) {
-    // bf16 tile -> eight 128-row x 64-column boxes over the (now idle) P slots, laid out
+    // bf16 tile -> eight 128-row x 64-column boxes in the (now idle) V ring, laid out
     // with the 128-byte swizzle, then TMA stores; the per-request 3-D tensor map
     // clips rows past the request's last node.
     for (int c = 0; c < 256 / 64; ++c) {
@@ -648,7 +629,7 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, cons
 #pragma unroll
         for (int k = 0; k < 64; ++k) v[k] = 0u;
       }
-      const uint32_t box = cx.base + P_OFF + (g * 4 + c) * CHUNK + (uint32_t)r * 128u;
+      const uint32_t box = cx.base + V_OFF + (g * 4 + c) * CHUNK + (uint32_t)r * 128u;
 #pragma unroll
       for (int q = 0; q < 8; ++q)
         st_shared_v4(box + ((q ^ (r & 7)) << 4),
@@ -659,8 +640,8 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, cons
     }
     fence_proxy_async_cta();
     named_bar_sync(1, GROUP);
-    if (threadIdx.x == 64 && ok && mt < p.mtiles) {
-      for (int bx = 0; bx < 8; ++bx) tma_store_3d(tm_o, cx.base + P_OFF + bx * CHUNK, bx * KC, mt * BM, b);
+    if (threadIdx.x == 64 && ok) {
+      for (int bx = 0; bx < 8; ++bx) tma_store_3d(tm_o, cx.base + V_OFF + bx * CHUNK, bx * KC, mt * BM, b);
       bulk_commit_group();
       bulk_wait_group_read0();
     }
@@ -697,7 +678,7 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, cons
 }
 
 // ====================================================================== kernel
-__global__ void __cluster_dims__(CLUSTER, 1, 1) __launch_bounds__(NTHREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant__ CUtensorMap tm_qr,
                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -710,16 +691,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   const uint32_t rank = cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int unit = (int)cluster_id_x();
-  const int mp = unit % p.mpairs;
-  const int sp = (unit / p.mpairs) % p.splits;
-  const int b = unit / (p.mpairs * p.splits);
-  const int mt = 2 * mp + (int)(rank & 1);           // this CTA's M tile (may be past the last)
-  const bool is_qk = rank < 2, leader = (rank & 1) == 0;
+  const int mt = unit % p.mtiles;
+  const int sp = (unit / p.mtiles) % p.splits;
+  const int b = unit / (p.mtiles * p.splits);
   const int n = p.n, H = p.H;
 
   const int64_t L = p.cache_lens[b];
-  if (L < 0 || L + n > p.cap) {          // all four CTAs see the same value and leave together
-    if (rank == 0 && threadIdx.x == 0 && mp == 0 && sp == 0) raise_dev_error(p.err, KD_DEV_CACHE_FULL);
+  if (L < 0 || L + n > p.cap) {          // both CTAs see the same value and leave together
+    if (rank == 0 && threadIdx.x == 0 && mt == 0 && sp == 0) raise_dev_error(p.err, KD_DEV_CACHE_FULL);
     return;
   }
   const int64_t nkeys = L + n;
@@ -733,22 +712,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   Ctx cx;
   cx.base = base;
   cx.abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + OFF_ABORT);
-  cx.rank = rank;
+  cx.peer = rank ^ 1u;
   cx.err = p.err;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBAR; ++i) {
       uint32_t cnt = 1;
-      if (i == CORR_DONE) cnt = GROUP;
-      if (i == QT_FULL || i == S_EMPTY) cnt = 2;
+      if (i == QT_FULL || i == S_EMPTY || i == CORR_DONE) cnt = GROUP;
+      if (i == STATS) cnt = 4;
       mbar_init(cx.bar(i), cnt);
     }
     *cx.abort_flag = 0u;
     fence_mbar_init();
   }
-  if (warp == 1) {                       // one TMEM allocation per pair, same columns in both CTAs
-    tmem_alloc_pair(base + OFF_TMEM, 512);
-    tmem_relinquish_pair();
+  if (warp == 1) {
+    tmem_alloc(base + OFF_TMEM, 512);
+    tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_qa);
@@ -763,12 +742,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + OFF_TMEM);
 
-  if (is_qk) {
+  if (rank == 0) {
     if (warp == 0) {
-      if (lane == 0 && ntiles > 0)
-        qk_producer(cx, &tm_qa, &tm_qr, &tm_c, &tm_r, qrow0, krow0, ntiles, leader);
+      if (lane == 0 && ntiles > 0) qk_producer(cx, &tm_qa, &tm_qr, &tm_c, &tm_r, qrow0, krow0, ntiles);
     } else if (warp == 1) {
-      if (lane == 0 && ntiles > 0 && leader) qk_mma(cx, tmem, ntiles);
+      if (lane == 0 && ntiles > 0) qk_mma(cx, tmem, ntiles);
       __syncwarp();
     } else {
       qk_softmax(cx, p, gbase, tmem, b, mt, sp, L, kbeg, ntiles);
@@ -788,7 +766,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem, 512);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -842,20 +820,20 @@ static int make_out_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t
   return KD_OK;
 }
 
-// Co-resident 4-CTA clusters of the kernel on the current device (cached).
-static int active_clusters(int sms) {
+// Co-resident 2-CTA clusters of the kernel on the current device (cached).
+static int active_pairs(int sms) {
   static int cached[64];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
-  int pairs = sms / CLUSTER;
+  int pairs = sms / 2;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(CLUSTER * pairs, 1, 1);
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(NTHREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cudaLaunchAttribute at;
   at.id = cudaLaunchAttributeClusterDimension;
-  at.val.clusterDim.x = CLUSTER;
+  at.val.clusterDim.x = 2;
   at.val.clusterDim.y = 1;
   at.val.clusterDim.z = 1;
   cfg.attrs = &at;
@@ -870,11 +848,11 @@ static int active_clusters(int sms) {
 }  // namespace tc
 
 // Split count for B requests of n nodes and H heads when the caller leaves it to
-// the library: minimise waves x (tiles per unit + fixed cost) over the clusters
-// that fit at once, with key length bounded by cap.  A unit is a pair of M tiles.
+// the library: minimise waves x (tiles per unit + fixed cost) over the pairs that
+// fit at once, with key length bounded by cap.
 int auto_splits(int B, int n, int H, int64_t cap, int pairs) {
   const int64_t mtiles = ((int64_t)n * H + tc::BM - 1) / tc::BM;
-  const int64_t units = (int64_t)B * ((mtiles + 1) / 2);
+  const int64_t units = (int64_t)B * mtiles;
   const int64_t T = (cap + tc::BQ - 1) / tc::BQ;
   int best = 1;
   double best_cost = 1e300;
@@ -902,7 +880,7 @@ using namespace kd;
 
 extern "C" size_t kd_verify_workspace_bytes(int B, int n, int H, int64_t cap, int kv_splits) {
   if (!shapes_ok(B, n) || H < 1 || H > KD_MAX_HEADS || cap < 1 || kv_splits < 0 || kv_splits > 64) return 0;
-  const int s = kv_splits > 0 ? kv_splits : auto_splits(B, n, H, cap, 37);
+  const int s = kv_splits > 0 ? kv_splits : auto_splits(B, n, H, cap, 74);
   return workspace_bytes_for(B, n, H, s);
 }
 
@@ -935,7 +913,7 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   }
   int splits = kv_splits;
   if (splits == 0) {
-    splits = auto_splits(B, n, H, cap, tc::active_clusters(sms));
+    splits = auto_splits(B, n, H, cap, tc::active_pairs(sms));
     while (splits > 1 && workspace_bytes_for(B, n, H, splits) > ws_bytes) --splits;
   }
   if (workspace_bytes_for(B, n, H, splits) > ws_bytes) return KD_ERANGE;
@@ -943,8 +921,8 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   CUtensorMap tq, tr, tcv, tkr, tv, to;
   if ((st = tc::make_map(&tq, q_abs, KD_D_C, (uint64_t)rows, KD_D_C * 2, tc::BM))) return st;
   if ((st = tc::make_map(&tr, q_rope, KD_D_R, (uint64_t)rows, KD_D_R * 2, tc::BM))) return st;
-  if ((st = tc::make_map(&tcv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::KH))) return st;
-  if ((st = tc::make_map(&tkr, k_rope, KD_D_R, (uint64_t)(B * cap), (uint64_t)sr * 2, tc::KH))) return st;
+  if ((st = tc::make_map(&tcv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::BQ))) return st;
+  if ((st = tc::make_map(&tkr, k_rope, KD_D_R, (uint64_t)(B * cap), (uint64_t)sr * 2, tc::BQ))) return st;
   if ((st = tc::make_map(&tv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::VKEYS))) return st;
   if ((st = tc::make_out_map(&to, out, (uint64_t)rows / B, (uint64_t)B))) return st;
 
@@ -965,13 +943,12 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   prm.H = H;
   prm.W = (n + 31) / 32;
   prm.mtiles = (int)((rows / B + tc::BM - 1) / tc::BM);
-  prm.mpairs = (prm.mtiles + 1) / 2;
   prm.splits = splits;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  const int64_t units = (int64_t)B * prm.mpairs * splits;
-  if (tc::CLUSTER * units > INT32_MAX) return KD_EINVAL;
-  tc::attn_tc_kernel<<<dim3((unsigned)(tc::CLUSTER * units)), tc::NTHREADS, tc::SMEM_BYTES, stream>>>(
-      tq, tr, tcv, tkr, tv, to, prm);
+  const int64_t units = (int64_t)B * prm.mtiles * splits;
+  if (2 * units > INT32_MAX) return KD_EINVAL;
+  tc::attn_tc_kernel<<<dim3((unsigned)(2 * units)), tc::NTHREADS, tc::SMEM_BYTES, stream>>>(tq, tr, tcv, tkr, tv, to,
+                                                                                         prm);
   st = launch_status("attn_tc_kernel");
   if (st || splits == 1) return st;
   return launch_combine(prm.part_o, prm.part_lse, cache_lens, B, n, H, cap, splits, out, lse, stream);
