@@ -73,8 +73,8 @@ constexpr int VG = 4 * VCH;             // one V group: 64 keys x 256 latent col
 constexpr int NVG = 4;                  // V ring depth
 constexpr int PBYTES = BM * BN * 2;     // one bf16 P tile (two 16 KB swizzle columns)
 constexpr int SLOT_ALPHA = PBYTES;      // f32 [128] per-row rescale factor
-constexpr int SLOT_COPY = PBYTES + 512; // bytes that reach the PV CTA per P tile
-constexpr int WARP_ROWS_BYTES = 32 * 128;  // one warp's 32 rows of one 64-key swizzle atom
+constexpr int SLOT_FLAG = PBYTES + 512; // u32 rescale-needed flag
+constexpr int SLOT_COPY = PBYTES + 528; // bytes moved to the PV CTA per tile
 constexpr int PSLOT = PBYTES + 1024;    // slot stride (keeps 1024-byte alignment)
 
 // TMEM columns of the QK CTA
@@ -196,26 +196,6 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) {     // MN-major, S
   return smem_desc_sw128(saddr, VCH, 1024);
 }
 
-// 2^y on the FMA pipe, used for a share of the softmax exponentials so that the
-// MUFU unit (16 results per cycle per SM) is not the only source.  Cody-Waite
-// style range reduction y = n + f with n = round(y), f in [-1/2, 1/2] (the
-// 1.5 * 2^23 addend rounds y to an integer in the low mantissa bits), a cubic for
-// 2^f, and n added to the result's exponent field.  The cubic is the
-// relative-error minimax fit of 2^f on [-1/2, 1/2] found by a Remez exchange:
-// max relative error 7.5e-5 (also when evaluated in fp32), far below the bf16
-// rounding that P undergoes next.  y is clamped at -127 so that -inf (a masked
-// key) gives exactly 0.
-__device__ __forceinline__ float exp2_fma(float y) {
-  y = fmaxf(y, -127.f);
-  const float t = y + 12582912.f;
-  const float f = y - (t - 12582912.f);
-  float q = fmaf(0.05517166905792616f, f, 0.2426111221932161f);
-  q = fmaf(q, f, 0.6932609854606553f);
-  q = fmaf(q, f, 0.9999280735394012f);
-  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
-}
-constexpr int FMA_EXP_EVERY = 4;        // every 4th column pair uses exp2_fma, the rest ex2.approx
-
 // Word q (0..3) of a node's visibility mask, without dynamic register indexing.
 __device__ __forceinline__ uint32_t mask_word(const uint32_t (&w)[4], int q) {
   return q == 0 ? w[0] : (q == 1 ? w[1] : (q == 2 ? w[2] : w[3]));
@@ -289,46 +269,37 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, uint32_t tmem, int ntiles)
   wait_bar(cx, cx.bar(DRAIN), 0);
 }
 
-// One 128-key half of a QK tile.  Each softmax warp works alone here: it
-// exponentiates its 32 rows x 64 columns (raw scores s, p = 2^(s * scale_log2 - m)),
-// adds them to the rows' running sums, writes them into its own contiguous 4 KB
-// slice of staging slot u % 2 (32 rows of one 64-key atom of the K-major,
-// 128-byte-swizzled P layout) and ships that slice with one bulk copy that
-// completes on the PV CTA's barrier.  Group 0 warps also ship the rows' rescale
-// factors.
-__device__ __forceinline__ bool emit_p(const Ctx& cx, uint8_t* gbase, const float (&s)[64], int u,
-                                       float scale_log2, float mb, float alpha, int r, int g,
-                                       int quad, uint32_t peer_p, uint32_t peer_ctrl, float& l_part) {
-  const int lane = threadIdx.x & 31;
+// One 128-key half of a QK tile: exponentiate this thread's 64 columns against
+// the row reference mb, add them to the running sum, and ship the bf16 P tile
+// (plus the per-row rescale factor for the PV side) through staging slot u % 2.
+__device__ __forceinline__ bool emit_p(const Ctx& cx, uint8_t* gbase, const float (&x)[64], int u,
+                                       float mb, float alpha, bool rescale_row, int r, int g,
+                                       uint32_t peer_p, uint32_t peer_ctrl, float& l_part) {
   const uint32_t sb = u & 1;
   float rs[4] = {0.f, 0.f, 0.f, 0.f};
   uint32_t pk[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
-    const float y0 = fmaf(s[2 * c], scale_log2, -mb), y1 = fmaf(s[2 * c + 1], scale_log2, -mb);
-    const bool fma_pipe = (c % FMA_EXP_EVERY) == FMA_EXP_EVERY - 1;
-    const float p0 = fma_pipe ? exp2_fma(y0) : ex2(y0);
-    const float p1 = fma_pipe ? exp2_fma(y1) : ex2(y1);
+    const float p0 = ex2(x[2 * c] - mb), p1 = ex2(x[2 * c + 1] - mb);
     rs[c & 3] += p0 + p1;
     pk[c] = pack_bf16x2(p0, p1);
   }
   l_part += (rs[0] + rs[1]) + (rs[2] + rs[3]);
   // staging slot sb (and the peer's P slot sb) is free once the PV MMAs of P tile u-2 completed
-  if (!wait_warp(cx, cx.bar(P_FREE + sb), ((u >> 1) & 1) ^ 1)) return false;
-  const uint32_t slice = (uint32_t)(g * (BM * 128) + quad * WARP_ROWS_BYTES);
+  if (!wait_group(cx, cx.bar(P_FREE + sb), ((u >> 1) & 1) ^ 1)) return false;
   const uint32_t stg = cx.base + STG_OFF + sb * PSLOT;
-  const uint32_t prow = stg + slice + (uint32_t)lane * 128u;
+  const uint32_t prow = stg + g * (BM * 128) + (uint32_t)r * 128u;
 #pragma unroll
   for (int q = 0; q < 8; ++q)
     st_shared_v4(prow + ((q ^ (r & 7)) << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-  if (g == 0) reinterpret_cast<float*>(gbase + STG_OFF + sb * PSLOT + SLOT_ALPHA)[r] = alpha;
+  float* stgf = reinterpret_cast<float*>(gbase + STG_OFF + sb * PSLOT);
+  if (g == 0) stgf[(SLOT_ALPHA >> 2) + r] = alpha;
   fence_proxy_async_cta();
-  __syncwarp();
-  if (lane == 0) {
-    const uint32_t dst = peer_p + sb * PSLOT, bar = peer_ctrl + 8u * P_FULL + 8u * sb;
-    bulk_copy_to_peer(dst + slice, stg + slice, WARP_ROWS_BYTES, bar);
-    if (g == 0)
-      bulk_copy_to_peer(dst + SLOT_ALPHA + quad * 128, stg + SLOT_ALPHA + quad * 128, 128, bar);
+  const bool any = named_bar_red_or(1, GROUP, rescale_row);
+  if (threadIdx.x == 64) {
+    reinterpret_cast<uint32_t*>(stgf)[SLOT_FLAG >> 2] = any ? 1u : 0u;
+    fence_proxy_async_cta();
+    bulk_copy_to_peer(peer_p + sb * PSLOT, stg, SLOT_COPY, peer_ctrl + 8u * P_FULL + 8u * sb);
   }
   return true;
 }
@@ -384,33 +355,26 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
   }
   const uint32_t peer_p = map_to_rank(cx.base + P_OFF, cx.peer);
   const uint32_t peer_ctrl = map_to_rank(cx.base, cx.peer);
-  const uint32_t pair_bar = 2 + quad;          // the two warps (one per group) that share rows
-  const float sl2 = p.scale_log2;
-  float m_ref = -INFINITY, l_part = 0.f;       // reference max in log2 units; partial row sum
+  float m_ref = -INFINITY, l_part = 0.f;
   bool ok = true;
-  for (int t = 0; t < ntiles; ++t) {
-    // a warp whose wait gave up still meets its partner warp at the pair barrier
-    // below, so both leave the loop together
-    const bool okw = ok && wait_warp(cx, cx.bar(S_FULL), t & 1);
-    // this thread's columns: keys 64 g .. 64 g + 63 of each 128-key half h of the tile (raw scores)
+  for (int t = 0; t < ntiles && ok; ++t) {
+    if (!(ok = wait_group(cx, cx.bar(S_FULL), t & 1))) break;
+    tc_fence_after();
+    // this thread's columns: keys 64 g .. 64 g + 63 of each 128-key half h of the tile
     float x[2][64];
-    if (okw) {
-      tc_fence_after();
+    {
       uint32_t u0[64], u1[64];
       tmem_ld64(lane_addr + TS + g * 64, u0);
       tmem_ld64(lane_addr + TS + BN + g * 64, u1);
       tmem_wait_ld();
 #pragma unroll
       for (int k = 0; k < 64; ++k) {
-        x[0][k] = __uint_as_float(u0[k]);
-        x[1][k] = __uint_as_float(u1[k]);
+        x[0][k] = __uint_as_float(u0[k]) * p.scale_log2;
+        x[1][k] = __uint_as_float(u1[k]) * p.scale_log2;
       }
-      tc_fence_before();
-      mbar_arrive(cx.bar(S_EMPTY));            // TMEM free for the next tile's MMAs
-    } else {
-#pragma unroll
-      for (int k = 0; k < 64; ++k) x[0][k] = x[1][k] = -INFINITY;
     }
+    tc_fence_before();
+    mbar_arrive(cx.bar(S_EMPTY));              // TMEM free for the next tile's MMAs
     // mask: only keys at or beyond L need it
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -433,35 +397,36 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
         mx[0] = fmaxf(mx[0], x[h][c]); mx[1] = fmaxf(mx[1], x[h][c + 1]);
         mx[2] = fmaxf(mx[2], x[h][c + 2]); mx[3] = fmaxf(mx[3], x[h][c + 3]);
       }
-    // row max over both groups' columns: exchange with the partner warp only
-    xch[g * BM + r] = max4(mx[0], mx[1], mx[2], mx[3]) * sl2;
-    if (named_bar_red_or(pair_bar, 64, !okw)) {
-      ok = false;
-      break;
-    }
+    xch[g * BM + r] = max4(mx[0], mx[1], mx[2], mx[3]);
+    named_bar_sync(1, GROUP);
     const float tmax = fmaxf(xch[r], xch[BM + r]);
-    named_bar_sync(pair_bar, 64);              // both reads done before the next write
     float alpha = 1.f;
+    bool rescale_row = false;
     if (tmax > m_ref + RESCALE_THRESHOLD) {
-      alpha = m_ref != -INFINITY ? ex2(m_ref - tmax) : 0.f;
+      if (m_ref != -INFINITY) {
+        alpha = ex2(m_ref - tmax);
+        rescale_row = true;
+      } else {
+        alpha = 0.f;
+      }
       l_part *= alpha;
       m_ref = tmax;
     }
     const float mb = m_ref == -INFINITY ? 0.f : m_ref;
-    ok = emit_p(cx, gbase, x[0], 2 * t, sl2, mb, alpha, r, g, quad, peer_p, peer_ctrl, l_part) &&
-         emit_p(cx, gbase, x[1], 2 * t + 1, sl2, mb, 1.f, r, g, quad, peer_p, peer_ctrl, l_part);
+    ok = emit_p(cx, gbase, x[0], 2 * t, mb, alpha, rescale_row, r, g, peer_p, peer_ctrl, l_part) &&
+         emit_p(cx, gbase, x[1], 2 * t + 1, mb, 1.f, false, r, g, peer_p, peer_ctrl, l_part);
   }
   // final row statistics for the epilogue: l = both groups' partial sums
+  named_bar_sync(1, GROUP);
   xch[g * BM + r] = l_part;
-  ok = !named_bar_red_or(pair_bar, 64, !ok);
+  named_bar_sync(1, GROUP);
   if (g == 0) {
     st_cluster_u32(peer_ctrl + OFF_MFIN + r * 4, __float_as_uint(m_ref));
     st_cluster_u32(peer_ctrl + OFF_LFIN + r * 4, __float_as_uint(xch[r] + xch[BM + r]));
-    __syncwarp();
-    if (lane == 0) mbar_arrive_remote(peer_ctrl + 8u * STATS);
   }
-  ok = !named_bar_red_or(1, GROUP, !ok);
+  named_bar_sync(1, GROUP);
   if (threadIdx.x == 64) {
+    mbar_arrive_remote(peer_ctrl + 8u * STATS);
     // the last P_FREE arrivals come from the peer's MMA completion: wait for them
     const int np = 2 * ntiles;
     if (ok)
@@ -502,16 +467,8 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, uint8_t* gbase, uint32_t t
     const uint32_t sb = t & 1;
     if (lane == 0) mbar_arrive_expect_tx(cx.bar(P_FULL + sb), SLOT_COPY);
     if (!(ok = wait_warp(cx, cx.bar(P_FULL + sb), (t >> 1) & 1, true))) break;
-    // rows whose reference max moved (alpha not 1; alpha 0 means the row had no
-    // visible key yet, so its O row is still 0) need O rescaled first
-    const volatile float* al = reinterpret_cast<const volatile float*>(gbase + P_OFF + sb * PSLOT + SLOT_ALPHA);
-    bool moved = false;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float a = al[lane * 4 + q];
-      moved |= (a != 1.f && a != 0.f);
-    }
-    const bool flag = __any_sync(0xffffffffu, moved);
+    const uint32_t flag =
+        *reinterpret_cast<volatile uint32_t*>(gbase + P_OFF + sb * PSLOT + SLOT_FLAG);
     if (flag && t > 0) {
       // every earlier PV MMA must be done before O is rescaled
       if (!(ok = wait_warp(cx, cx.bar(PV_TILE), (t - 1) & 1))) break;
@@ -719,7 +676,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
     for (int i = 0; i < NBAR; ++i) {
       uint32_t cnt = 1;
       if (i == QT_FULL || i == S_EMPTY || i == CORR_DONE) cnt = GROUP;
-      if (i == STATS) cnt = 4;
       mbar_init(cx.bar(i), cnt);
     }
     *cx.abort_flag = 0u;
