@@ -109,6 +109,8 @@ constexpr int OFF_EVTILE = 524;         // u32 P slot of a rescale event        
 constexpr int OFF_MFIN = 2048;          // f32 [128] final running max (log2)      [PV, remote]
 constexpr int OFF_LFIN = 2560;          // f32 [128] final running sum             [PV, remote]
 constexpr int OFF_XCH = 3072;           // f32 [2][128] max / sum exchange         [QK, local]
+constexpr int OFF_ORDER = 1024;         // i32 [LPT_MAX] requests by length, at start only
+constexpr int LPT_MAX = 256;            // longest-first dispatch for up to this many requests
 static_assert(NBAR * 8 <= OFF_TMEM, "barrier block overflow");
 
 constexpr int Q_OFF = CTRL;                           // Q chunk 8 (rope)
@@ -650,7 +652,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   const int unit = (int)cluster_id_x();
   const int mt = unit % p.mtiles;
   const int sp = (unit / p.mtiles) % p.splits;
-  const int b = unit / (p.mtiles * p.splits);
+  // Clusters are dispatched in index order; handing the longest requests out first
+  // (their units stay adjacent, so their M tiles share K/V in L2) keeps the last
+  // wave short when cache lengths differ.  Each CTA ranks the requests itself.
+  int b = unit / (p.mtiles * p.splits);
+  if (p.B > 1 && p.B <= LPT_MAX) {
+    int* order = reinterpret_cast<int*>(gbase + OFF_ORDER);
+    for (int i = threadIdx.x; i < p.B; i += blockDim.x) {
+      const int li = p.cache_lens[i];
+      int pos = 0;
+      for (int j = 0; j < p.B; ++j) {
+        const int lj = p.cache_lens[j];
+        pos += (lj > li) || (lj == li && j < i);
+      }
+      order[pos] = i;
+    }
+    __syncthreads();
+    b = order[b];
+    __syncthreads();
+  }
   const int n = p.n, H = p.H;
 
   const int64_t L = p.cache_lens[b];
