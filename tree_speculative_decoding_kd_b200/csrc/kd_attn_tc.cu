@@ -438,12 +438,20 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
 }
 
 // ====================================================================== PV CTA roles
+// Keys of P tile t, key group kh that exist (the rest of the last QK tile lies past
+// the request's last key).  Groups with none are neither loaded nor multiplied.
+__device__ __forceinline__ int group_keys(int64_t kbeg, int64_t nkeys, int t, int kh) {
+  const int64_t left = nkeys - (kbeg + (int64_t)t * BN + kh * VKEYS);
+  return left <= 0 ? 0 : (left < VKEYS ? (int)left : VKEYS);
+}
+
 __device__ __forceinline__ void pv_producer(const Ctx& cx, const CUtensorMap* tm_v, int64_t krow0,
-                                            int ntiles) {
+                                            int64_t kbeg, int64_t nkeys, int ntiles) {
   bool ok = true;
   uint32_t gi = 0;
   for (int t = 0; t < 2 * ntiles && ok; ++t) {
     for (int kh = 0; kh < BN / VKEYS && ok; ++kh) {
+      if (group_keys(kbeg, nkeys, t, kh) == 0) continue;
       const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN + kh * VKEYS);
       for (int hh = 0; hh < 2; ++hh, ++gi) {
         const uint32_t gs = gi % NVG, k = gi / NVG;
@@ -483,22 +491,21 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, uint8_t* gbase, uint32_t t
       ++nres;
     }
     tc_fence_after();
-    const int64_t kt = kbeg + (int64_t)t * BN;
-    const int nvalid = (int)((nkeys - kt) < BN ? (nkeys - kt) : BN);
     for (int kh = 0; kh < BN / VKEYS && ok; ++kh) {
-      const int nv = min(max(nvalid - kh * VKEYS, 0), VKEYS);
+      const int nv = group_keys(kbeg, nkeys, t, kh);
+      if (nv == 0) continue;             // P is zero there: nothing to add (and nothing loaded)
       for (int hh = 0; hh < 2 && ok; ++hh, ++gi) {
         const uint32_t gs = gi % NVG;
         if (!(ok = wait_warp(cx, cx.bar(V_FULL + gs), (gi / NVG) & 1u))) break;
         if (nv < VKEYS) {
           // rows past the request's last key may hold anything (even NaN bit
-          // patterns); P is 0 there but 0 * NaN is not, so clear them
+          // patterns); P is 0 there but 0 * NaN is not, so clear them.  A key row is
+          // 128 contiguous bytes of its 64-column box (the swizzle stays inside a row).
           uint4* vg = reinterpret_cast<uint4*>(gbase + V_OFF + gs * VG);
-          const int per_chunk = (VKEYS - nv) * 8;
-          for (int idx = lane; idx < 4 * per_chunk; idx += 32) {
-            const int q = idx / per_chunk, e = idx % per_chunk;
-            vg[q * (VCH / 16) + nv * 8 + e] = make_uint4(0u, 0u, 0u, 0u);
-          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            for (int e = nv * 8 + lane; e < VKEYS * 8; e += 32)
+              vg[q * (VCH / 16) + e] = make_uint4(0u, 0u, 0u, 0u);
           fence_proxy_async_cta();
           __syncwarp();
         }
@@ -532,7 +539,7 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, uint8_t* gbase, uint32_t t
 
 // Correction / epilogue groups: thread (g, r) owns row r, O columns [256 g, 256 g + 256).
 __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, const CUtensorMap* tm_o,
-                                            uint8_t* gbase, uint32_t tmem, int b, int mt, int sp,
+                                            const CUtensorMap* tm_po, uint8_t* gbase, uint32_t tmem, int b, int mt, int sp,
                                             int ntiles) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = (warp - 2) >> 2;
@@ -574,7 +581,7 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, cons
   const float inv = l > 0.f ? 1.f / l : 0.f;
   const bool have_o = ntiles > 0;
   const int64_t grow = (int64_t)b * rows_req + R;
-  const int64_t prow = ((int64_t)sp * p.B * rows_req) + grow;
+  const int64_t prow = ((int64_t)sp * p.B * rows_req) + grow;     // row of part_lse
   if (p.splits == 1) {
     // bf16 tile -> eight 128-row x 64-column boxes in the (now idle) V ring, laid out
     // with the 128-byte swizzle, then TMA stores; the per-request 3-D tensor map
@@ -605,26 +612,44 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, cons
       bulk_wait_group_read0();
     }
   } else {
-    uint32_t v0[32], v1[32];
-    for (int c = 0; c < 256 / 64; ++c) {
-      if (have_o && ok) {
-        tmem_ld32(lane_addr + c * 64, v0);
-        tmem_ld32(lane_addr + c * 64 + 32, v1);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int k = 0; k < 32; ++k) v0[k] = v1[k] = 0u;
+    // f32 partial tile in two rounds of eight 128-row x 32-column boxes (128-byte
+    // swizzle) in the V ring; round k covers columns [256 g + 128 k, +128) of each
+    // group.  The 3-D map [splits x B][rows][512] clips rows past the last node.
+    for (int k = 0; k < 2; ++k) {
+      if (k == 1) {
+        if (threadIdx.x == 64 && ok) bulk_wait_group_read0();
+        named_bar_sync(1, GROUP);
       }
-      if (!valid) continue;
-      const int col = g * 256 + c * 64;
-      float4* dst = reinterpret_cast<float4*>(p.part_o + prow * KD_D_C + col);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[64];
+        if (have_o && ok) {
+          tmem_ld64(lane_addr + k * 128 + h * 64, v);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int o = q * 4;
-        dst[q] = make_float4(__uint_as_float(v0[o]) * inv, __uint_as_float(v0[o + 1]) * inv,
-                             __uint_as_float(v0[o + 2]) * inv, __uint_as_float(v0[o + 3]) * inv);
-        dst[8 + q] = make_float4(__uint_as_float(v1[o]) * inv, __uint_as_float(v1[o + 1]) * inv,
-                                 __uint_as_float(v1[o + 2]) * inv, __uint_as_float(v1[o + 3]) * inv);
+          for (int i = 0; i < 64; ++i) v[i] = 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint32_t box = cx.base + V_OFF + (g * 4 + h * 2 + j) * CHUNK + (uint32_t)r * 128u;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int o = j * 32 + q * 4;
+            st_shared_v4(box + ((q ^ (r & 7)) << 4), __float_as_uint(__uint_as_float(v[o]) * inv),
+                         __float_as_uint(__uint_as_float(v[o + 1]) * inv),
+                         __float_as_uint(__uint_as_float(v[o + 2]) * inv),
+                         __float_as_uint(__uint_as_float(v[o + 3]) * inv));
+          }
+        }
+      }
+      fence_proxy_async_cta();
+      named_bar_sync(1, GROUP);
+      if (threadIdx.x == 64 && ok) {
+        for (int bx = 0; bx < 8; ++bx)
+          tma_store_3d(tm_po, cx.base + V_OFF + bx * CHUNK, (bx >> 2) * 256 + k * 128 + (bx & 3) * 32,
+                       mt * BM, sp * p.B + b);
+        bulk_commit_group();
+        if (k == 1) bulk_wait_group_read0();
       }
     }
   }
@@ -641,7 +666,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant__ CUtensorMap tm_qr,
                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-               const __grid_constant__ Params p) {
+               const __grid_constant__ CUtensorMap tm_po, const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -712,6 +737,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
     tma_prefetch_desc(&tm_r);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_o);
+    if (p.splits > 1) tma_prefetch_desc(&tm_po);
   }
   tc_fence_before();
   cluster_sync();
@@ -729,15 +755,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
     }
   } else {
     if (warp == 0) {
-      if (lane == 0) pv_producer(cx, &tm_v, krow0, ntiles);
+      if (lane == 0) pv_producer(cx, &tm_v, krow0, kbeg, nkeys, ntiles);
     } else if (warp == 1) {
       pv_mma(cx, gbase, tmem, kbeg, nkeys, ntiles);
     } else {
-      pv_epilogue(cx, p, &tm_o, gbase, tmem, b, mt, sp, ntiles);
+      pv_epilogue(cx, p, &tm_o, &tm_po, gbase, tmem, b, mt, sp, ntiles);
     }
   }
 
   // ------------------------------------------------------- teardown
+  __syncwarp();          // the roles leave lanes behind (single-lane issuers, lane 64's waits)
   __syncthreads();
   cluster_sync();
   if (warp == 1) {
@@ -791,6 +818,25 @@ static int make_out_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t
                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled(out)");
+    return KD_ELAUNCH;
+  }
+  return KD_OK;
+}
+
+// 3-D f32 view [splits x B][rows][512] of the split partials, 32 x 128 x 1 boxes,
+// 128-byte swizzle.
+static int make_part_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t zs) {
+  auto fn = encode_fn();
+  if (!fn) return KD_ELAUNCH;
+  cuuint64_t dims[3] = {KD_D_C, rows, zs};
+  cuuint64_t strides[2] = {KD_D_C * 4, rows * KD_D_C * 4};
+  cuuint32_t box[3] = {32, BM, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled(partial)");
     return KD_ELAUNCH;
   }
   return KD_OK;
@@ -894,7 +940,7 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   }
   if (workspace_bytes_for(B, n, H, splits) > ws_bytes) return KD_ERANGE;
 
-  CUtensorMap tq, tr, tcv, tkr, tv, to;
+  CUtensorMap tq, tr, tcv, tkr, tv, to, tpo;
   if ((st = tc::make_map(&tq, q_abs, KD_D_C, (uint64_t)rows, KD_D_C * 2, tc::BM))) return st;
   if ((st = tc::make_map(&tr, q_rope, KD_D_R, (uint64_t)rows, KD_D_R * 2, tc::BM))) return st;
   if ((st = tc::make_map(&tcv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::BQ))) return st;
@@ -921,10 +967,15 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   prm.mtiles = (int)((rows / B + tc::BM - 1) / tc::BM);
   prm.splits = splits;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  if (splits > 1) {
+    if ((st = tc::make_part_map(&tpo, prm.part_o, (uint64_t)rows / B, (uint64_t)splits * B))) return st;
+  } else {
+    tpo = to;                                   // not read with one split
+  }
   const int64_t units = (int64_t)B * prm.mtiles * splits;
   if (2 * units > INT32_MAX) return KD_EINVAL;
-  tc::attn_tc_kernel<<<dim3((unsigned)(2 * units)), tc::NTHREADS, tc::SMEM_BYTES, stream>>>(tq, tr, tcv, tkr, tv, to,
-                                                                                         prm);
+  tc::attn_tc_kernel<<<dim3((unsigned)(2 * units)), tc::NTHREADS, tc::SMEM_BYTES, stream>>>(
+      tq, tr, tcv, tkr, tv, to, tpo, prm);
   st = launch_status("attn_tc_kernel");
   if (st || splits == 1) return st;
   return launch_combine(prm.part_o, prm.part_lse, cache_lens, B, n, H, cap, splits, out, lse, stream);
