@@ -271,19 +271,23 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, uint32_t tmem, int ntiles)
   wait_bar(cx, cx.bar(DRAIN), 0);
 }
 
-// One 128-key half of a QK tile: exponentiate this thread's 64 columns against
-// the row reference mb, add them to the running sum, and ship the bf16 P tile
-// (plus the per-row rescale factor for the PV side) through staging slot u % 2.
+// One 128-key half of a QK tile: exponentiate this thread's 64 raw scores x as
+// 2^(x s - mb) (s = softmax scale in log2 units, mb the scaled row reference),
+// add them to the running sum, and ship the bf16 P tile (plus the per-row rescale
+// factor for the PV side) through staging slot u % 2.
 __device__ __forceinline__ bool emit_p(const Ctx& cx, uint8_t* gbase, const float (&x)[64], int u,
-                                       float mb, float alpha, bool rescale_row, int r, int g,
+                                       float s, float mb, float alpha, bool rescale_row, int r, int g,
                                        uint32_t peer_p, uint32_t peer_ctrl, float& l_part) {
   const uint32_t sb = u & 1;
   float rs[4] = {0.f, 0.f, 0.f, 0.f};
   uint32_t pk[32];
+  const float nmb = -mb;
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
-    const float p0 = ex2(x[2 * c] - mb), p1 = ex2(x[2 * c + 1] - mb);
-    rs[c & 3] += p0 + p1;
+    float a0, a1;
+    ffma2(a0, a1, x[2 * c], x[2 * c + 1], s, nmb);
+    const float p0 = ex2(a0), p1 = ex2(a1);
+    fadd2(rs[2 * (c & 1)], rs[2 * (c & 1) + 1], p0, p1);
     pk[c] = pack_bf16x2(p0, p1);
   }
   l_part += (rs[0] + rs[1]) + (rs[2] + rs[3]);
@@ -370,9 +374,9 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
       tmem_ld64(lane_addr + TS + BN + g * 64, u1);
       tmem_wait_ld();
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        x[0][k] = __uint_as_float(u0[k]) * p.scale_log2;
-        x[1][k] = __uint_as_float(u1[k]) * p.scale_log2;
+      for (int k = 0; k < 64; ++k) {            // raw scores: the scale is applied in emit_p
+        x[0][k] = __uint_as_float(u0[k]);
+        x[1][k] = __uint_as_float(u1[k]);
       }
     }
     tc_fence_before();
@@ -391,17 +395,20 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
         }
       }
     }
+    // row max of the raw scores (the scale is positive, so it commutes with max)
     float mx[4] = {x[0][0], x[0][1], x[0][2], x[0][3]};
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int c = (h == 0 ? 4 : 0); c < 64; c += 4) {
-        mx[0] = fmaxf(mx[0], x[h][c]); mx[1] = fmaxf(mx[1], x[h][c + 1]);
-        mx[2] = fmaxf(mx[2], x[h][c + 2]); mx[3] = fmaxf(mx[3], x[h][c + 3]);
+      for (int c = 0; c < 64; c += 8) {              // (re-reading x[0][0..3] is harmless)
+        mx[0] = fmax3(mx[0], x[h][c], x[h][c + 4]);
+        mx[1] = fmax3(mx[1], x[h][c + 1], x[h][c + 5]);
+        mx[2] = fmax3(mx[2], x[h][c + 2], x[h][c + 6]);
+        mx[3] = fmax3(mx[3], x[h][c + 3], x[h][c + 7]);
       }
     xch[g * BM + r] = max4(mx[0], mx[1], mx[2], mx[3]);
     named_bar_sync(1, GROUP);
-    const float tmax = fmaxf(xch[r], xch[BM + r]);
+    const float tmax = fmaxf(xch[r], xch[BM + r]) * p.scale_log2;
     float alpha = 1.f;
     bool rescale_row = false;
     if (tmax > m_ref + RESCALE_THRESHOLD) {
@@ -415,8 +422,9 @@ __device__ __forceinline__ void qk_softmax(const Ctx& cx, const Params& p, uint8
       m_ref = tmax;
     }
     const float mb = m_ref == -INFINITY ? 0.f : m_ref;
-    ok = emit_p(cx, gbase, x[0], 2 * t, mb, alpha, rescale_row, r, g, peer_p, peer_ctrl, l_part) &&
-         emit_p(cx, gbase, x[1], 2 * t + 1, mb, 1.f, false, r, g, peer_p, peer_ctrl, l_part);
+    ok = emit_p(cx, gbase, x[0], 2 * t, p.scale_log2, mb, alpha, rescale_row, r, g, peer_p, peer_ctrl,
+                l_part) &&
+         emit_p(cx, gbase, x[1], 2 * t + 1, p.scale_log2, mb, 1.f, false, r, g, peer_p, peer_ctrl, l_part);
   }
   // final row statistics for the epilogue: l = both groups' partial sums
   named_bar_sync(1, GROUP);
