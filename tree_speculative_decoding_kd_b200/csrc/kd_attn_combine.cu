@@ -29,18 +29,30 @@ combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_
   for (int k = 0; k < 16; ++k) acc[k] = 0.f;
   float sum = 0.f;
   if (mx != -INFINITY) {
-    for (int s = 0; s < splits; ++s) {
-      const float ls = part_lse[(int64_t)s * rows + row];
-      const float wgt = ptx::ex2((ls - mx) * LOG2E);     // 0 for an empty partition
-      sum += wgt;
-      const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)s * rows + row) * KD_D_C + lane * 16);
+    // four partitions at a time: all of their loads are issued before any is used,
+    // so a row's partials stream in together rather than one round trip per partition
+    for (int s0 = 0; s0 < splits; s0 += 4) {
+      float4 v[4][4];
+      float wgt[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 v = src[q];
-        acc[4 * q + 0] = fmaf(wgt, v.x, acc[4 * q + 0]);
-        acc[4 * q + 1] = fmaf(wgt, v.y, acc[4 * q + 1]);
-        acc[4 * q + 2] = fmaf(wgt, v.z, acc[4 * q + 2]);
-        acc[4 * q + 3] = fmaf(wgt, v.w, acc[4 * q + 3]);
+      for (int j = 0; j < 4; ++j) {
+        const int s = s0 + j < splits ? s0 + j : s0;        // past the end: reload s0 at weight 0
+        const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)s * rows + row) * KD_D_C + lane * 16);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[j][q] = src[q];
+        const float ls = part_lse[(int64_t)s * rows + row];
+        wgt[j] = s0 + j < splits ? ptx::ex2((ls - mx) * LOG2E) : 0.f;   // 0 for an empty partition
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        sum += wgt[j];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[4 * q + 0] = fmaf(wgt[j], v[j][q].x, acc[4 * q + 0]);
+          acc[4 * q + 1] = fmaf(wgt[j], v[j][q].y, acc[4 * q + 1]);
+          acc[4 * q + 2] = fmaf(wgt[j], v[j][q].z, acc[4 * q + 2]);
+          acc[4 * q + 3] = fmaf(wgt[j], v[j][q].w, acc[4 * q + 3]);
+        }
       }
     }
   }
