@@ -44,3 +44,22 @@ def tree_accept_batch(node_tokens, parents, target_argmax):
         ln[b] = l
         bonus[b] = t
     return path, ln, bonus
+
+
+def target_argmax(logits):
+    """The target's greedy token after each node: the index of the largest logit in its
+    row ("The Architecture of Pragmatic Ambition", section "The Output Knowledge: What
+    This Message Creates": argmax is an engine primitive, and the speculative output must
+    equal greedy decoding token for token).  Readings for what the pages leave open:
+    among equal maxima the lowest index wins, a NaN ranks above every number (the first
+    NaN wins), and -0.0 equals +0.0.  numpy's argmax is exactly this definition.
+    logits [..., V] -> int32 [...]."""
+    return np.argmax(np.asarray(logits), axis=-1).astype(np.int32)
+
+
+def tree_accept_logits(node_tokens, parents, logits):
+    """Greedy acceptance fed by the target argmax of fp32 logits [B][n][V]:
+    returns (argmax [B][n], path, len, bonus) as tree_accept_batch."""
+    am = target_argmax(logits)
+    path, ln, bonus = tree_accept_batch(node_tokens, parents, am)
+    return am, path, ln, bonus

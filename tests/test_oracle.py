@@ -7,6 +7,9 @@
   scipy's logsumexp; closed forms (equal scores); softmax invariants.
 * accept: brute-force enumeration of root-to-node paths on small trees; the
   planted path the generator knows; budget 0.
+* target argmax: an explicit comparison loop over small rows full of ties, signed
+  zeros, infinities and NaNs; hand-written special cases; the token the generator
+  planted in each row of full-vocabulary logits.
 * compaction: slot-by-slot expectations, including an overlap where copying in
   the wrong order gives a different cache.
 """
@@ -19,7 +22,7 @@ import scipy.special
 import torch
 
 import oracle
-from oracle.accept import tree_accept_batch
+from oracle.accept import target_argmax, tree_accept_batch, tree_accept_logits
 from tree_speculative_decoding_kd_b200 import workload as W
 
 RNG = np.random.default_rng(1234)
@@ -382,3 +385,49 @@ def test_golden_tiny_regression():
     np.testing.assert_allclose(now["lse"], g["lse"], rtol=0, atol=1e-12)
     np.testing.assert_allclose(now["out_node_sums"], g["out_node_sums"], rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(now["out_00_first8"], g["out_00_first8"], rtol=1e-12, atol=1e-16)
+
+
+# ---------------------------------------------------------------- target argmax
+def _argmax_loop(row):
+    """The definition spelled out: scan left to right, keep the first maximum, a NaN beats
+    every number and the first NaN is kept (Python's > treats -0.0 and +0.0 as equal)."""
+    best_i, best = 0, float(row[0])
+    for i in range(1, len(row)):
+        if math.isnan(best):
+            break
+        x = float(row[i])
+        if math.isnan(x) or x > best:
+            best_i, best = i, x
+    return best_i
+
+
+def test_argmax_matches_comparison_loop():
+    vals = np.array([-2.0, -1.0, -0.0, 0.0, 1.0, 2.0, np.inf, -np.inf, np.nan], dtype=np.float32)
+    rng = np.random.default_rng(77)
+    for _ in range(400):
+        V = int(rng.integers(1, 24))
+        p = rng.random(len(vals))
+        p[-1] *= 0.1                     # NaNs are rarer, so many rows have none
+        row = rng.choice(vals, size=V, p=p / p.sum()).astype(np.float32)
+        assert int(target_argmax(row)) == _argmax_loop(row), row
+
+
+@pytest.mark.parametrize("row, want", [
+    ([-0.0, 0.0], 0), ([0.0, -0.0], 0), ([1.0, np.nan, np.nan], 1), ([-np.inf, -np.inf], 0),
+    ([np.inf, np.nan], 1), ([3.0, 5.0, 5.0, 4.0], 1), ([7.0], 0),
+    ([np.float32(1e-45), 0.0], 0), ([-1e-45, -0.0], 1),
+])
+def test_argmax_special_cases(row, want):
+    assert int(target_argmax(np.array(row, dtype=np.float32))) == want
+
+
+def test_accept_logits_recovers_planted_paths():
+    wl = W.make_workload("tiny")
+    st = wl.step
+    lg = W.draw_logits(wl.cfg, st)
+    am, path, ln, bonus = tree_accept_logits(st.tokens, st.parents, lg)
+    assert (am == st.argmax).all()
+    for b in range(wl.cfg.B):
+        assert list(path[b, :ln[b]]) == [int(x) for x in st.planted[b]]
+    p2, l2, b2 = tree_accept_batch(st.tokens, st.parents, st.argmax)
+    assert (path == p2).all() and (ln == l2).all() and (bonus == b2).all()

@@ -1,7 +1,7 @@
 """Seeded synthetic workloads for the tree-verify step.
 
-This module only draws inputs: random latents, queries, trees, draft tokens and
-target argmaxes.  It computes nothing of the method itself (no attention, no
+This module only draws inputs: random latents, queries, trees, draft tokens,
+target argmaxes and target logits that carry them.  It computes nothing of the method itself (no attention, no
 acceptance walk, no compaction).  Both the CUDA path (through the Python
 binding) and the float64 oracle consume what it returns.
 
@@ -310,6 +310,25 @@ def draw_cache(cfg: Config, cache_lens: np.ndarray, fill: int) -> tuple[np.ndarr
             c_kv[b, :rows] = latent_bf16((rows, D_C), (cfg.seed, 6, b), pool=pool)
             k_rope[b, :rows] = latent_bf16((rows, D_R), (cfg.seed, 7, b), pool=pool)
     return c_kv, k_rope
+
+
+LOGIT_NOISE_CLIP = 6.0     # noise logits lie in [-6, 6] ...
+LOGIT_PLANTED = 7.0        # ... so the planted token is each row's unique maximum
+
+
+def draw_logits(cfg: Config, st: StepInputs, step: int = 0, vocab: int = VOCAB) -> np.ndarray:
+    """Target logits fp32 [B][n][vocab]: clipped N(0,1) noise with the step's planted
+    target token (st.argmax) set above the clip, so that the greedy token after each
+    node is the planted one."""
+    if int(st.argmax.max()) >= vocab:
+        raise ValueError("the step's tokens were drawn from a larger vocabulary")
+    g = np.random.default_rng([cfg.seed, 5, step])
+    B, n = st.parents.shape
+    lg = g.standard_normal((B, n, vocab), dtype=np.float32)
+    np.clip(lg, -LOGIT_NOISE_CLIP, LOGIT_NOISE_CLIP, out=lg)
+    bi, ni = np.meshgrid(np.arange(B), np.arange(n), indexing="ij")
+    lg[bi, ni, st.argmax] = LOGIT_PLANTED
+    return lg
 
 
 def make_workload(name_or_cfg, step: int = 0, **tree_override) -> Workload:
