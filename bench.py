@@ -265,6 +265,48 @@ def attn_extras(kd, torch, peaks, flush):
             ["tiny", "kimi_single", "batched", "long"]}
 
 
+def accept_logits_case(kd, torch, peaks, name="loop", reps=10, warm=3):
+    """Target argmax fused with greedy accept (kd_tree_accept_logits) on one step of a
+    configuration's trees with full-vocabulary fp32 logits; HBM bound (logits read once,
+    larger than L2, so no flush is needed)."""
+    wl = W.make_workload(name)
+    st = wl.step
+    logits = torch.from_numpy(W.draw_logits(wl.cfg, st)).cuda()
+    tok = torch.from_numpy(st.tokens).cuda()
+    par = torch.from_numpy(st.parents).cuda()
+    B, n, V = logits.shape
+    ws = kd.new_accept_workspace(B, n)
+    am = torch.empty(B, n, dtype=torch.int32, device="cuda")
+    path = torch.empty(B, n, dtype=torch.int32, device="cuda")
+    ln = torch.empty(B, dtype=torch.int32, device="cuda")
+    bonus = torch.empty(B, dtype=torch.int32, device="cuda")
+
+    def call():
+        kd.kd_tree_accept_logits(tok, par, logits, am, path, ln, bonus, ws)
+
+    for _ in range(warm):
+        call()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3)
+    ok = bool((am.cpu().numpy() == st.argmax).all())
+    t = float(np.median(times))
+    nbytes = B * n * V * 4
+    del logits
+    torch.cuda.empty_cache()
+    return {"workload": f"{name}: {B} requests x {n} nodes x {V} fp32 logits", "us": round(t * 1e6, 2),
+            "us_min": round(min(times) * 1e6, 2), "hbm_gbs": round(nbytes / t / 1e9, 1),
+            "roofline_frac": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 3), "bound": "hbm",
+            "bytes": nbytes, "planted_tokens_recovered": ok,
+            "timing": "CUDA events around each call; logits larger than L2, so no flush"}
+
+
 def run_attn_only(args):
     """--attn-only NAME: time just the attention of one configuration (profiling aid)."""
     import torch
@@ -370,10 +412,12 @@ def run_kd(args):
     e2e_rate = HN.whole_job_rate(args.steps, world, e2e_el)
 
     extras = None
+    next_rows = None
     cpu = None
     if rank == 0 and world == 1:
         if not args.no_extras:
             extras = attn_extras(kd, torch, peaks, HN.L2Flush("cuda"))
+            next_rows = {"accept_logits": accept_logits_case(kd, torch, peaks)}
         if not args.no_cpu_baseline:
             cpu = cpu_baseline(cfg, wl, host_steps[0])
 
@@ -412,6 +456,8 @@ def run_kd(args):
             line["cpu_baseline"] = cpu
         if extras is not None:
             line["per_config_attention"] = extras
+        if next_rows is not None:
+            line["next_rows"] = next_rows
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():

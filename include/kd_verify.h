@@ -17,6 +17,9 @@
  *                            tree ancestors;
  *   4. kd_tree_accept        greedy walk to the longest path matching the target
  *                            argmax ("The Knowledge Architecture");
+ *      kd_tree_accept_logits the same walk fed by the argmax of the target's
+ *                            logits, both in one launch ("The Output Knowledge:
+ *                            What This Message Creates");
  *   5. kd_kv_compact         the accepted path's latents, root included, gathered
  *                            into contiguous slots and the length advanced
  *                            ("The Reasoning That Preceded the Header"; read-all-
@@ -197,6 +200,38 @@ int kd_tree_verify_attn_noalloc(const kd_bf16_t* q_nope_absorbed, const kd_bf16_
 int kd_tree_accept(const int32_t* node_tokens, const int32_t* parents,
                    const int32_t* target_argmax, int B, int n, int32_t* path,
                    int32_t* len, int32_t* bonus, int32_t* dev_error, cudaStream_t stream);
+
+/*
+ * kd_accept_workspace_bytes -- scratch bytes kd_tree_accept_logits needs for B
+ * requests of n nodes (0 for invalid shapes).
+ */
+size_t kd_accept_workspace_bytes(int B, int n);
+
+/*
+ * kd_tree_accept_logits -- the target's greedy token after every node, taken from
+ * its logits, fused with kd_tree_accept in one launch ("The Architecture of
+ * Pragmatic Ambition", section "The Output Knowledge: What This Message Creates":
+ * argmax is an engine primitive, and the speculative output must equal greedy
+ * decoding token for token).
+ *   logits [B][n][V] fp32, row pitch V, 16-byte aligned, V a multiple of 4 and
+ *          at most 2^31 - 1 (V = 163840 for Kimi-K2).  Row (b, i) holds the
+ *          target's logits after node i.
+ *   target_argmax [B][n] int32 out, or NULL: index of the largest logit of each
+ *          row; the lowest index among equal maxima, a NaN above every number
+ *          (the first NaN wins), -0.0 equal to +0.0.
+ *   node_tokens, parents, path, len, bonus: as kd_tree_accept, with these tokens.
+ *   workspace: caller-owned device scratch of at least
+ *          kd_accept_workspace_bytes(B, n) bytes, 16-byte aligned, cleared by the
+ *          call; do not share it between calls that may overlap.
+ * Returns KD_EINVAL for null or misaligned pointers, bad shapes or V; KD_ERANGE
+ * if ws_bytes is too small.  A bad parent array sets KD_DEV_BAD_PARENT as
+ * kd_tree_accept does.  The logits are read once (streaming loads).
+ */
+int kd_tree_accept_logits(const int32_t* node_tokens, const int32_t* parents,
+                          const float* logits, int B, int n, int64_t V,
+                          int32_t* target_argmax, int32_t* path, int32_t* len,
+                          int32_t* bonus, void* workspace, size_t ws_bytes,
+                          int32_t* dev_error, cudaStream_t stream);
 
 /*
  * kd_kv_compact -- gather each request's accepted latents into contiguous slots.

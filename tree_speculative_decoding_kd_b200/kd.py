@@ -37,6 +37,8 @@ _SIGS = {
     "kd_tree_verify_attn_noalloc": (_i, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _i,
                                          _f, _p, _p, _i, _p, _p]),
     "kd_tree_accept": (_i, [_p, _p, _p, _i, _i, _p, _p, _p, _p, _p]),
+    "kd_accept_workspace_bytes": (_sz, [_i, _i]),
+    "kd_tree_accept_logits": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _p, _p, _p, _sz, _p, _p]),
     "kd_kv_compact": (_i, [_p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _p, _p]),
     "kd_kv_write_nodes": (_i, [_p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _p, _p]),
     "kd_read_device_error": (_i, [_p, _i, _p]),
@@ -182,6 +184,38 @@ def kd_tree_verify_attn_simt(q_abs, q_rope, c_kv, k_rope, cache_lens, vis, posit
                                         _ptr(dev_error), _stream(stream)),
            "kd_tree_verify_attn_simt")
     return out, lse
+
+
+def new_accept_workspace(B, n, device=None) -> torch.Tensor:
+    nbytes = int(lib.kd_accept_workspace_bytes(B, n))
+    if nbytes == 0:
+        raise KdError("kd_accept_workspace_bytes: invalid shapes")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def kd_tree_accept_logits(node_tokens, parents, logits, target_argmax=None, path=None,
+                          length=None, bonus=None, workspace=None, dev_error=None, stream=None):
+    """Target argmax of fp32 logits [B][n][V] fused with greedy acceptance.
+    Returns (target_argmax, path, len, bonus)."""
+    for t, nm in ((node_tokens, "node_tokens"), (parents, "parents")):
+        _need(t, torch.int32, nm)
+    _need(logits, torch.float32, "logits")
+    B, n = parents.shape
+    if logits.dim() != 3 or tuple(logits.shape[:2]) != (B, n):
+        raise ValueError("logits must be [B][n][V]")
+    V = logits.shape[2]
+    dev = parents.device
+    if target_argmax is None:
+        target_argmax = torch.empty(B, n, dtype=torch.int32, device=dev)
+    path = torch.empty(B, n, dtype=torch.int32, device=dev) if path is None else path
+    length = torch.empty(B, dtype=torch.int32, device=dev) if length is None else length
+    bonus = torch.empty(B, dtype=torch.int32, device=dev) if bonus is None else bonus
+    workspace = new_accept_workspace(B, n, dev) if workspace is None else workspace
+    _check(lib.kd_tree_accept_logits(_ptr(node_tokens), _ptr(parents), _ptr(logits), B, n, V,
+                                     _ptr(target_argmax), _ptr(path), _ptr(length), _ptr(bonus),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _ptr(dev_error), _stream(stream)), "kd_tree_accept_logits")
+    return target_argmax, path, length, bonus
 
 
 def kd_tree_accept(node_tokens, parents, target_argmax, path=None, length=None, bonus=None,
