@@ -10,7 +10,7 @@ from tree_speculative_decoding_kd_b200 import workload as W
 
 pytestmark = pytest.mark.gpu
 
-CHUNK = 8192          # logits per CTA in the kernel; ties are planted across this boundary
+CHUNK = 16384         # logits per CTA in the kernel; ties are planted across this boundary
 
 
 def dev_i32(a):

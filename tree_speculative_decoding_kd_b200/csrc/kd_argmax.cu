@@ -9,12 +9,15 @@
 //       matches those tokens.
 //
 // Reading logits [B][n][V] once is the whole cost (HBM bound: 4·V bytes per node).
-// One CTA streams one 32 KB chunk of one node's row with coalesced 16-byte loads,
-// eight in flight per thread, and reduces it to a 64-bit rank: the value's
-// order-preserving key in the high word, the complement of the index in the low
-// word, so that one unsigned max picks the largest value and, among equal values,
-// the lowest index.  NaN ranks above every number (the first NaN wins) and -0.0
-// ranks as +0.0.  The chunk's rank is merged into the row's by atomicMax; the
+// One CTA streams one 64 KB chunk of one node's row with coalesced 16-byte loads,
+// sixteen in flight per thread.  Each thread keeps its 64 values in registers, takes
+// their NaN-propagating max (one instruction per value) and then scans them from the
+// highest index down for the value equal to that max (or for a NaN), so that the last
+// hit is the lowest index; -0.0 == +0.0 there.  Only then does it form a 64-bit rank:
+// the value's order-preserving key in the high word, the complement of the index in
+// the low word, so that one unsigned max across threads picks the largest value and,
+// among equal values, the lowest index.  NaN ranks above every number and -0.0 ranks
+// as +0.0.  The chunk's rank is merged into the row's by atomicMax; the
 // last CTA of a request (counted per request) turns the n ranks into tokens and
 // runs the greedy walk with one warp.
 
@@ -24,8 +27,8 @@
 namespace kd {
 
 constexpr int AM_THREADS = 256;
-constexpr int AM_VEC = 8;                                  // 16-byte loads per thread per chunk
-constexpr int AM_CHUNK = AM_THREADS * AM_VEC * 4;          // 8192 logits = 32 KB per CTA
+constexpr int AM_VEC = 16;                                 // 16-byte loads per thread per chunk
+constexpr int AM_CHUNK = AM_THREADS * AM_VEC * 4;          // 16384 logits = 64 KB per CTA
 
 // Rank of logit x at index idx (see above).
 __device__ __forceinline__ unsigned long long logit_rank(float x, uint32_t idx) {
@@ -38,6 +41,12 @@ __device__ __forceinline__ unsigned long long logit_rank(float x, uint32_t idx) 
     key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);      // monotone in the value
   }
   return ((unsigned long long)key << 32) | (unsigned long long)(0xffffffffu - idx);
+}
+
+__device__ __forceinline__ float max_nan3(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
@@ -57,26 +66,35 @@ argmax_accept_kernel(const float* __restrict__ logits, int64_t V, int chunks, in
   const float4* src = reinterpret_cast<const float4*>(logits + row * V);
   const int64_t e0 = (int64_t)chunk * AM_CHUNK + (int64_t)threadIdx.x * 4;
 
-  // all eight loads first, then the ranks (V is a multiple of 4, so a vector is
-  // either wholly inside the row or wholly past its end)
+  // all eight loads first (V is a multiple of 4, so a vector is either wholly inside
+  // the row or wholly past its end; past the end reads as -inf and is never chosen)
+  const float NEG = -INFINITY;
   float4 x[AM_VEC];
 #pragma unroll
   for (int j = 0; j < AM_VEC; ++j) {
     const int64_t e = e0 + (int64_t)j * AM_THREADS * 4;
-    x[j] = e < V ? __ldcs(src + (e >> 2)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    x[j] = e < V ? __ldcs(src + (e >> 2)) : make_float4(NEG, NEG, NEG, NEG);
   }
-  unsigned long long m = 0ull;                             // below every real rank
+  float mv = x[0].x;
 #pragma unroll
-  for (int j = 0; j < AM_VEC; ++j) {
+  for (int j = 0; j < AM_VEC; ++j) mv = max_nan3(max_nan3(mv, x[j].x, x[j].y), x[j].z, x[j].w);
+  // lowest index holding mv (or the first NaN): scan down, the last hit wins
+  const bool want_nan = mv != mv;
+  const bool whole = e0 + (int64_t)(AM_VEC - 1) * AM_THREADS * 4 < V;   // no element past V
+  uint32_t idx = 0xffffffffu;
+#pragma unroll
+  for (int j = AM_VEC - 1; j >= 0; --j) {
     const int64_t e = e0 + (int64_t)j * AM_THREADS * 4;
-    if (e < V) {
-      const uint32_t i = (uint32_t)e;
-      m = umax64(m, logit_rank(x[j].x, i));
-      m = umax64(m, logit_rank(x[j].y, i + 1));
-      m = umax64(m, logit_rank(x[j].z, i + 2));
-      m = umax64(m, logit_rank(x[j].w, i + 3));
+    const bool in = whole || e < V;
+    const uint32_t i = (uint32_t)e;
+    const float v[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+#pragma unroll
+    for (int c = 3; c >= 0; --c) {
+      const bool hit = want_nan ? (v[c] != v[c]) : (v[c] == mv);
+      idx = (hit && in) ? i + c : idx;
     }
   }
+  unsigned long long m = idx == 0xffffffffu ? 0ull : logit_rank(mv, idx);   // 0: below every rank
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = umax64(m, __shfl_xor_sync(0xffffffffu, m, off));
   __shared__ unsigned long long wm[AM_THREADS / 32];
