@@ -61,6 +61,10 @@ def parse():
     ap.add_argument("--attn-only", default=None, choices=["tiny", "kimi_single", "batched", "long"],
                     help="time only the attention of one single-step configuration")
     ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--accept-logits-only", action="store_true",
+                    help="time only the fused target argmax + accept on the loop workload's trees")
+    ap.add_argument("--requests", type=int, default=0,
+                    help="with --accept-logits-only: use the first R requests (0 = all)")
     return ap.parse_args()
 
 
@@ -265,15 +269,16 @@ def attn_extras(kd, torch, peaks, flush):
             ["tiny", "kimi_single", "batched", "long"]}
 
 
-def accept_logits_case(kd, torch, peaks, name="loop", reps=10, warm=3):
+def accept_logits_case(kd, torch, peaks, name="loop", reps=10, warm=3, requests=0):
     """Target argmax fused with greedy accept (kd_tree_accept_logits) on one step of a
     configuration's trees with full-vocabulary fp32 logits; HBM bound (logits read once,
-    larger than L2, so no flush is needed)."""
+    larger than L2 at the loop workload's 64 requests, so no flush is needed)."""
     wl = W.make_workload(name)
     st = wl.step
-    logits = torch.from_numpy(W.draw_logits(wl.cfg, st)).cuda()
-    tok = torch.from_numpy(st.tokens).cuda()
-    par = torch.from_numpy(st.parents).cuda()
+    R = requests or wl.cfg.B
+    logits = torch.from_numpy(W.draw_logits(wl.cfg, st)[:R]).cuda()
+    tok = torch.from_numpy(st.tokens[:R]).cuda()
+    par = torch.from_numpy(st.parents[:R]).cuda()
     B, n, V = logits.shape
     ws = kd.new_accept_workspace(B, n)
     am = torch.empty(B, n, dtype=torch.int32, device="cuda")
@@ -295,7 +300,7 @@ def accept_logits_case(kd, torch, peaks, name="loop", reps=10, warm=3):
         e1.record()
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1) * 1e-3)
-    ok = bool((am.cpu().numpy() == st.argmax).all())
+    ok = bool((am.cpu().numpy() == st.argmax[:R]).all())
     t = float(np.median(times))
     nbytes = B * n * V * 4
     del logits
@@ -305,6 +310,16 @@ def accept_logits_case(kd, torch, peaks, name="loop", reps=10, warm=3):
             "roofline_frac": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 3), "bound": "hbm",
             "bytes": nbytes, "planted_tokens_recovered": ok,
             "timing": "CUDA events around each call; logits larger than L2, so no flush"}
+
+
+def run_accept_logits_only(args):
+    """--accept-logits-only: time just kd_tree_accept_logits (profiling aid)."""
+    import torch
+    torch.cuda.set_device(0)
+    from tree_speculative_decoding_kd_b200 import kd
+    peaks = HN.load_peaks(ROOT)
+    res = accept_logits_case(kd, torch, peaks, reps=args.reps, warm=1, requests=args.requests)
+    print(json.dumps({"accept_logits_only": True, **res}), flush=True)
 
 
 def run_attn_only(args):
@@ -466,6 +481,9 @@ def run_kd(args):
 
 def main():
     args = parse()
+    if args.accept_logits_only:
+        run_accept_logits_only(args)
+        return
     if args.attn_only:
         run_attn_only(args)
     elif args.impl == "reference":

@@ -10,14 +10,14 @@
 //
 // Reading logits [B][n][V] once is the whole cost (HBM bound: 4·V bytes per node).
 // One CTA streams one 64 KB chunk of one node's row with coalesced 16-byte loads,
-// sixteen in flight per thread.  Each thread keeps its 64 values in registers, takes
-// their NaN-propagating max (one instruction per value) and then scans them from the
-// highest index down for the value equal to that max (or for a NaN), so that the last
-// hit is the lowest index; -0.0 == +0.0 there.  Only then does it form a 64-bit rank:
-// the value's order-preserving key in the high word, the complement of the index in
-// the low word, so that one unsigned max across threads picks the largest value and,
-// among equal values, the lowest index.  NaN ranks above every number and -0.0 ranks
-// as +0.0.  The chunk's rank is merged into the row's by atomicMax; the
+// sixteen in flight per thread.  Each thread keeps its 64 values in registers and
+// takes their NaN-propagating max (a third of an instruction per value); the CTA then
+// agrees on the chunk's maximum, and only the threads that hold it scan their values
+// from the highest index down for it (or for a NaN), so that the last hit is the
+// lowest index; -0.0 == +0.0 there.  Ranks compare as 64-bit words: the value's
+// order-preserving key in the high word, the complement of the index in the low word,
+// so that one unsigned max picks the largest value and, among equal values, the
+// lowest index.  NaN ranks above every number and -0.0 ranks as +0.0.  The chunk's rank is merged into the row's by atomicMax; the
 // last CTA of a request (counted per request) turns the n ranks into tokens and
 // runs the greedy walk with one warp.
 
@@ -30,17 +30,12 @@ constexpr int AM_THREADS = 256;
 constexpr int AM_VEC = 16;                                 // 16-byte loads per thread per chunk
 constexpr int AM_CHUNK = AM_THREADS * AM_VEC * 4;          // 16384 logits = 64 KB per CTA
 
-// Rank of logit x at index idx (see above).
-__device__ __forceinline__ unsigned long long logit_rank(float x, uint32_t idx) {
+// Order-preserving key of a logit (see above).
+__device__ __forceinline__ uint32_t logit_key(float x) {
   uint32_t u = __float_as_uint(x);
-  uint32_t key;
-  if ((u & 0x7fffffffu) > 0x7f800000u) {
-    key = 0xffffffffu;                                     // NaN: above every number
-  } else {
-    if (u == 0x80000000u) u = 0u;                          // -0.0 ranks as +0.0
-    key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);      // monotone in the value
-  }
-  return ((unsigned long long)key << 32) | (unsigned long long)(0xffffffffu - idx);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return 0xffffffffu;   // NaN: above every number
+  if (u == 0x80000000u) u = 0u;                              // -0.0 ranks as +0.0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);         // monotone in the value
 }
 
 __device__ __forceinline__ float max_nan3(float a, float b, float c) {
@@ -53,7 +48,7 @@ __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsig
   return a > b ? a : b;
 }
 
-__global__ void __launch_bounds__(AM_THREADS)
+__global__ void __launch_bounds__(AM_THREADS, 3)
 argmax_accept_kernel(const float* __restrict__ logits, int64_t V, int chunks, int n,
                      const int32_t* __restrict__ tokens, const int32_t* __restrict__ parents,
                      int32_t* argmax, unsigned long long* best, unsigned int* done,
@@ -78,27 +73,41 @@ argmax_accept_kernel(const float* __restrict__ logits, int64_t V, int chunks, in
   float mv = x[0].x;
 #pragma unroll
   for (int j = 0; j < AM_VEC; ++j) mv = max_nan3(max_nan3(mv, x[j].x, x[j].y), x[j].z, x[j].w);
-  // lowest index holding mv (or the first NaN): scan down, the last hit wins
-  const bool want_nan = mv != mv;
-  const bool whole = e0 + (int64_t)(AM_VEC - 1) * AM_THREADS * 4 < V;   // no element past V
-  uint32_t idx = 0xffffffffu;
+  // the chunk's maximum key (a thread whose elements all lie past V holds -inf, which
+  // only wins if every real element is -inf too, and then the scan below skips it)
+  uint32_t k = logit_key(mv);
 #pragma unroll
-  for (int j = AM_VEC - 1; j >= 0; --j) {
-    const int64_t e = e0 + (int64_t)j * AM_THREADS * 4;
-    const bool in = whole || e < V;
-    const uint32_t i = (uint32_t)e;
-    const float v[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
-#pragma unroll
-    for (int c = 3; c >= 0; --c) {
-      const bool hit = want_nan ? (v[c] != v[c]) : (v[c] == mv);
-      idx = (hit && in) ? i + c : idx;
-    }
-  }
-  unsigned long long m = idx == 0xffffffffu ? 0ull : logit_rank(mv, idx);   // 0: below every rank
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = umax64(m, __shfl_xor_sync(0xffffffffu, m, off));
+  for (int off = 16; off > 0; off >>= 1) k = max(k, __shfl_xor_sync(0xffffffffu, k, off));
+  __shared__ uint32_t wk[AM_THREADS / 32];
   __shared__ unsigned long long wm[AM_THREADS / 32];
   __shared__ int last;
+  if (lane == 0) wk[warp] = k;
+  __syncthreads();
+  uint32_t kmax = wk[0];
+#pragma unroll
+  for (int w = 1; w < AM_THREADS / 32; ++w) kmax = max(kmax, wk[w]);
+  // only threads holding it look for its lowest index: scan down, the last hit wins
+  unsigned long long m = 0ull;                             // below every real rank
+  if (logit_key(mv) == kmax) {
+    const bool want_nan = mv != mv;
+    const bool whole = e0 + (int64_t)(AM_VEC - 1) * AM_THREADS * 4 < V;   // no element past V
+    uint32_t idx = 0xffffffffu;
+#pragma unroll
+    for (int j = AM_VEC - 1; j >= 0; --j) {
+      const int64_t e = e0 + (int64_t)j * AM_THREADS * 4;
+      const bool in = whole || e < V;
+      const uint32_t i = (uint32_t)e;
+      const float v[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+#pragma unroll
+      for (int c = 3; c >= 0; --c) {
+        const bool hit = want_nan ? (v[c] != v[c]) : (v[c] == mv);
+        idx = (hit && in) ? i + c : idx;
+      }
+    }
+    if (idx != 0xffffffffu) m = ((unsigned long long)kmax << 32) | (unsigned long long)(0xffffffffu - idx);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = umax64(m, __shfl_xor_sync(0xffffffffu, m, off));
   if (lane == 0) wm[warp] = m;
   __syncthreads();
   if (warp != 0) return;
