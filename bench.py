@@ -58,7 +58,7 @@ def parse():
     ap.add_argument("--impl", choices=["kd", "reference"], default="kd")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-config attention lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--attn-only", default=None, choices=["tiny", "kimi_single", "batched", "long"],
+    ap.add_argument("--attn-only", default=None, choices=["tiny", "kimi_single", "batched", "long", "extend"],
                     help="time only the attention of one single-step configuration")
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--accept-logits-only", action="store_true",
@@ -432,7 +432,8 @@ def run_kd(args):
     if rank == 0 and world == 1:
         if not args.no_extras:
             extras = attn_extras(kd, torch, peaks, HN.L2Flush("cuda"))
-            next_rows = {"accept_logits": accept_logits_case(kd, torch, peaks)}
+            next_rows = {"accept_logits": accept_logits_case(kd, torch, peaks),
+                         "causal_extend": attn_case(kd, torch, peaks, HN.L2Flush("cuda"), "extend")}
         if not args.no_cpu_baseline:
             cpu = cpu_baseline(cfg, wl, host_steps[0])
 

@@ -397,6 +397,27 @@ def test_attn_full_size_sampled(kd, name):
     assert_attn(out, lse, ro, rl, f"{name} full")
 
 
+def test_causal_extend_chunk_full_size_sampled(kd):
+    """Chunked causal extend (a chain tree of 128 nodes) through the verify kernel: 4
+    requests over 16384-token caches; the oracle computes three nodes of every request,
+    the first and the last included."""
+    wl = W.make_workload("extend")
+    assert (wl.step.parents[:, 1:] == np.arange(127)).all()
+    out, lse, bits = run_attn(kd, wl)
+    ro, rl = oracle_attn(wl, nodes=_sample_nodes(wl.cfg, np.random.default_rng(6)))
+    assert bits == 0
+    assert_attn(out, lse, ro, rl, "extend full")
+
+
+def test_causal_extend_chunk_small_exact(kd):
+    """A ragged 128-token causal chunk over a 300-token cache, every node checked."""
+    wl = W.make_workload(small("extend", B=1, H=16, L_lo=300, L_hi=300))
+    out, lse, bits = run_attn(kd, wl)
+    ro, rl = oracle_attn(wl)
+    assert bits == 0
+    assert_attn(out, lse, ro, rl, "extend small")
+
+
 def test_loop_full_size_two_steps(kd):
     """Config 5 exactly (64 requests, cap 18101): two whole steps, caches and
     lengths bit-exact, attention on sampled nodes."""

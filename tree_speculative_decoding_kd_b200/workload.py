@@ -78,6 +78,9 @@ CONFIGS = {
     "long": Config("long", 8, 64, 65, 32768, 32768, "depth", 12, 3),
     # 64 requests, L ~ U{2048..16384}, budget 16, 100 verify+accept+compact steps
     "loop": Config("loop", 64, 64, 17, 2048, 16384, "depth", 8, 4, steps=100),
+    # chunked causal extend through the same kernel: a chain "tree" (parent[i] = i - 1)
+    # makes the visibility mask causal; 4 requests extend a 16384-token cache by 128 tokens
+    "extend": Config("extend", 4, 64, 128, 16384, 16384, "chain", 0, 5),
 }
 
 # --------------------------------------------------------------------------
