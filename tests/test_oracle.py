@@ -10,6 +10,10 @@
 * target argmax: an explicit comparison loop over small rows full of ties, signed
   zeros, infinities and NaNs; hand-written special cases; the token the generator
   planted in each row of full-vocabulary logits.
+* tree build: brute-force enumeration of every path of small candidate sets (the
+  n - 1 best by score); chain (K = 1), star (D = 1) and all-ties (breadth-first)
+  special cases; structural invariants (topological parents, scores as exact float32
+  sums along the path, tokens of the right candidates).
 * compaction: slot-by-slot expectations, including an overlap where copying in
   the wrong order gives a different cache.
 """
@@ -431,3 +435,69 @@ def test_accept_logits_recovers_planted_paths():
         assert list(path[b, :ln[b]]) == [int(x) for x in st.planted[b]]
     p2, l2, b2 = tree_accept_batch(st.tokens, st.parents, st.argmax)
     assert (path == p2).all() and (ln == l2).all() and (bonus == b2).all()
+
+
+# ---------------------------------------------------------------- tree build
+from oracle.tree_build import tree_build  # noqa: E402
+
+
+def _draw_cands(rng, D, K, vocab=1000):
+    logp = np.sort(np.log(rng.dirichlet(np.ones(K), size=D)).astype(np.float32), axis=1)[:, ::-1]
+    toks = np.stack([rng.choice(vocab, K, replace=False) for _ in range(D)]).astype(np.int32)
+    return np.ascontiguousarray(logp), toks
+
+
+def _check_structure(par, tok, dep, sc, logp, toks, root):
+    assert par[0] == -1 and tok[0] == root and dep[0] == 0 and sc[0] == 0
+    for i in range(1, len(par)):
+        p = par[i]
+        assert 0 <= p < i and dep[i] == dep[p] + 1
+        j = int(np.nonzero(toks[dep[i] - 1] == tok[i])[0][0])
+        assert sc[i] == np.float32(sc[p] + logp[dep[i] - 1, j])      # exact float32 sum
+        assert sc[i] <= sc[i - 1] or dep[i] > dep[i - 1]              # pop order
+
+
+def test_tree_build_matches_brute_force_top_paths():
+    rng = np.random.default_rng(9)
+    for _ in range(60):
+        D, K = int(rng.integers(1, 5)), int(rng.integers(1, 4))
+        logp, toks = _draw_cands(rng, D, K)
+        total = sum(K ** d for d in range(1, D + 1))
+        n = int(rng.integers(1, total + 2))
+        # every path (j_1..j_d) with its float32 score summed in path order
+        paths = []
+        for d in range(1, D + 1):
+            for js in itertools.product(range(K), repeat=d):
+                s = np.float32(0.0)
+                for t, j in enumerate(js):
+                    s = np.float32(s + logp[t, j])
+                paths.append((s, js))
+        paths.sort(key=lambda x: (-float(x[0]), len(x[1]), x[1]))
+        want = {js for _, js in paths[: n - 1]}
+        par, tok, dep, sc = tree_build(logp, toks, 7, n)
+        _check_structure(par, tok, dep, sc, logp, toks, 7)
+        got = set()
+        for i in range(1, n):
+            js, k = [], i
+            while k > 0:
+                js.append(int(np.nonzero(toks[dep[k] - 1] == tok[k])[0][0]))
+                k = par[k]
+            got.add(tuple(reversed(js)))
+        assert got == want
+
+
+def test_tree_build_chain_star_and_ties():
+    rng = np.random.default_rng(3)
+    logp, toks = _draw_cands(rng, 6, 1)                     # K = 1: a chain
+    par, tok, dep, _ = tree_build(logp, toks, 5, 7)
+    assert list(par) == [-1, 0, 1, 2, 3, 4, 5] and list(dep) == list(range(7))
+    logp, toks = _draw_cands(rng, 1, 5)                     # D = 1: a star, best first
+    par, tok, dep, _ = tree_build(logp, toks, 5, 6)
+    assert list(par) == [-1, 0, 0, 0, 0, 0] and list(tok[1:]) == list(toks[0])
+    zero = np.zeros((3, 2), np.float32)                     # all ties: breadth first
+    toks = np.arange(6, dtype=np.int32).reshape(3, 2)
+    par, tok, dep, _ = tree_build(zero, toks, 9, 8)
+    assert list(par) == [-1, 0, 0, 1, 1, 2, 2, 3]
+    assert list(tok) == [9, 0, 1, 2, 3, 2, 3, 4]
+    with pytest.raises(ValueError):                         # too few candidate nodes
+        tree_build(zero[:1, :1], toks[:1, :1], 9, 3)
