@@ -312,6 +312,29 @@ def accept_logits_case(kd, torch, peaks, name="loop", reps=10, warm=3, requests=
             "timing": "CUDA events around each call; logits larger than L2, so no flush"}
 
 
+def tree_build_case(kd, torch, name="loop", depth=16, k=8, reps=20, warm=3):
+    """Best-first draft-tree build for every request of a configuration from drafter
+    candidates (depth x k per request); launch-latency sized (one warp per request)."""
+    cfg = W.CONFIGS[name]
+    logp, toks, root = W.draw_candidates(cfg, depth=depth, k=k)
+    lp, tk, rt = (torch.from_numpy(a).cuda() for a in (logp, toks, root))
+    for _ in range(warm):
+        kd.kd_tree_build(lp, tk, rt, cfg.n)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        kd.kd_tree_build(lp, tk, rt, cfg.n)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3)
+    return {"workload": f"{name}: {cfg.B} requests, {cfg.n} nodes from {depth} depths x {k} candidates",
+            "us": round(float(np.median(times)) * 1e6, 2), "us_min": round(min(times) * 1e6, 2),
+            "bound": "latency (one warp per request, one pop per node)",
+            "timing": "CUDA events around each call (includes the binding's output allocations)"}
+
+
 def run_accept_logits_only(args):
     """--accept-logits-only: time just kd_tree_accept_logits (profiling aid)."""
     import torch
@@ -433,7 +456,8 @@ def run_kd(args):
         if not args.no_extras:
             extras = attn_extras(kd, torch, peaks, HN.L2Flush("cuda"))
             next_rows = {"accept_logits": accept_logits_case(kd, torch, peaks),
-                         "causal_extend": attn_case(kd, torch, peaks, HN.L2Flush("cuda"), "extend")}
+                         "causal_extend": attn_case(kd, torch, peaks, HN.L2Flush("cuda"), "extend"),
+                         "tree_build": tree_build_case(kd, torch)}
         if not args.no_cpu_baseline:
             cpu = cpu_baseline(cfg, wl, host_steps[0])
 

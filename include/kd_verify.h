@@ -7,6 +7,8 @@
  *                            root first ("The Architectural Keystone: Writing the
  *                            Model Header ...", "The Reasoning That Preceded the
  *                            Header");
+ *   0. kd_tree_build         the draft tree itself, best first from the drafter's
+ *                            per-depth candidates ("The Knowledge Architecture");
  *   2. kd_tree_build_mask    per-node ancestor bitmasks from the parent array
  *                            ("The Architecture of Pragmatic Ambition", "The
  *                            Knowledge Architecture": attention over the tree with
@@ -184,6 +186,29 @@ int kd_tree_verify_attn_noalloc(const kd_bf16_t* q_nope_absorbed, const kd_bf16_
                                 const int32_t* positions, int B, int n, int H, float scale,
                                 kd_bf16_t* out, float* lse, int kv_splits, int32_t* dev_error,
                                 cudaStream_t stream);
+
+/*
+ * kd_tree_build -- best-first draft trees from per-depth drafter candidates, one per
+ * request ("The Architecture of Pragmatic Ambition", section "The Knowledge
+ * Architecture": the tree builder takes per-depth top-k candidates and constructs a
+ * best-first tree).  The pages give no scoring rule; this is the reading taken:
+ *   logp        [B][D][K] fp32: log-probabilities of depth d's K candidates, sorted
+ *               from the most to the least likely (not checked; unsorted input gives
+ *               the same deterministic steps, not a best-first tree); no NaN.
+ *   cand_tokens [B][D][K] int32: the candidates' tokens.
+ *   root_tokens [B] int32: the last verified token (node 0).
+ *   A node's score is the float32 sum of log-probabilities along its path.  The
+ *   tree is node 0 plus the n - 1 best nodes, popped best first from the frontier
+ *   of the tree so far (ties: lower depth, then lower parent, then lower
+ *   candidate); node index = pop order, so parents[i] < i.
+ *   parents, tokens [B][n] int32 out (parents[b][0] = -1); depth [B][n] int32 and
+ *   score [B][n] fp32 out, each optional (NULL).
+ * Limits: 1 <= n <= 128, 1 <= D <= 4096, 1 <= K <= 255, and the candidates must
+ * hold at least n - 1 nodes (K + K^2 + ... + K^D >= n - 1); otherwise KD_EINVAL.
+ */
+int kd_tree_build(const float* logp, const int32_t* cand_tokens, const int32_t* root_tokens,
+                  int B, int D, int K, int n, int32_t* parents, int32_t* tokens, int32_t* depth,
+                  float* score, cudaStream_t stream);
 
 /*
  * kd_tree_accept -- greedy acceptance of B verified trees.

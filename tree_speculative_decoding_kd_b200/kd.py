@@ -38,6 +38,7 @@ _SIGS = {
                                          _f, _p, _p, _i, _p, _p]),
     "kd_tree_accept": (_i, [_p, _p, _p, _i, _i, _p, _p, _p, _p, _p]),
     "kd_accept_workspace_bytes": (_sz, [_i, _i]),
+    "kd_tree_build": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p]),
     "kd_tree_accept_logits": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _p, _p, _p, _sz, _p, _p]),
     "kd_kv_compact": (_i, [_p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _p, _p]),
     "kd_kv_write_nodes": (_i, [_p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _p, _p]),
@@ -184,6 +185,26 @@ def kd_tree_verify_attn_simt(q_abs, q_rope, c_kv, k_rope, cache_lens, vis, posit
                                         _ptr(dev_error), _stream(stream)),
            "kd_tree_verify_attn_simt")
     return out, lse
+
+
+def kd_tree_build(logp, cand_tokens, root_tokens, n, stream=None):
+    """Best-first draft trees: logp fp32 [B][D][K] (sorted per depth), cand_tokens int32
+    [B][D][K], root_tokens int32 [B] -> (parents, tokens, depth, score), each [B][n]."""
+    _need(logp, torch.float32, "logp")
+    _need(cand_tokens, torch.int32, "cand_tokens")
+    _need(root_tokens, torch.int32, "root_tokens")
+    B, D, K = logp.shape
+    if tuple(cand_tokens.shape) != (B, D, K) or tuple(root_tokens.shape) != (B,):
+        raise ValueError("cand_tokens must be [B][D][K] and root_tokens [B]")
+    dev = logp.device
+    parents = torch.empty(B, n, dtype=torch.int32, device=dev)
+    tokens = torch.empty(B, n, dtype=torch.int32, device=dev)
+    depth = torch.empty(B, n, dtype=torch.int32, device=dev)
+    score = torch.empty(B, n, dtype=torch.float32, device=dev)
+    _check(lib.kd_tree_build(_ptr(logp), _ptr(cand_tokens), _ptr(root_tokens), B, D, K, n,
+                             _ptr(parents), _ptr(tokens), _ptr(depth), _ptr(score), _stream(stream)),
+           "kd_tree_build")
+    return parents, tokens, depth, score
 
 
 def new_accept_workspace(B, n, device=None) -> torch.Tensor:

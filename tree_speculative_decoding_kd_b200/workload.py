@@ -1,7 +1,7 @@
 """Seeded synthetic workloads for the tree-verify step.
 
 This module only draws inputs: random latents, queries, trees, draft tokens,
-target argmaxes and target logits that carry them.  It computes nothing of the method itself (no attention, no
+target argmaxes and target logits that carry them, and drafter candidates.  It computes nothing of the method itself (no attention, no
 acceptance walk, no compaction).  Both the CUDA path (through the Python
 binding) and the float64 oracle consume what it returns.
 
@@ -313,6 +313,20 @@ def draw_cache(cfg: Config, cache_lens: np.ndarray, fill: int) -> tuple[np.ndarr
             c_kv[b, :rows] = latent_bf16((rows, D_C), (cfg.seed, 6, b), pool=pool)
             k_rope[b, :rows] = latent_bf16((rows, D_R), (cfg.seed, 7, b), pool=pool)
     return c_kv, k_rope
+
+
+def draw_candidates(cfg: Config, step: int = 0, depth: int = 16, k: int = 8, vocab: int = VOCAB):
+    """Drafter candidates for the tree builder: per request and depth, k distinct tokens
+    with log-probabilities of a Dirichlet(1) draw, sorted from the most likely; and one
+    root token per request.  Returns (logp float32 [B][depth][k], tokens int32
+    [B][depth][k], root int32 [B])."""
+    g = np.random.default_rng([cfg.seed, 6, step])
+    p = g.dirichlet(np.ones(k), size=(cfg.B, depth))
+    logp = np.sort(np.log(p).astype(np.float32), axis=2)[:, :, ::-1].copy()
+    toks = np.stack([np.stack([g.choice(vocab, k, replace=False) for _ in range(depth)])
+                     for _ in range(cfg.B)]).astype(np.int32)
+    root = g.integers(0, vocab, size=cfg.B).astype(np.int32)
+    return logp, toks, root
 
 
 LOGIT_NOISE_CLIP = 6.0     # noise logits lie in [-6, 6] ...
