@@ -16,6 +16,9 @@
   sums along the path, tokens of the right candidates).
 * compaction: slot-by-slot expectations, including an overlap where copying in
   the wrong order gives a different cache.
+* paged caches: the logical view against an explicit per-slot loop over the page
+  table; identity page tables reduce to the contiguous functions; writes land only
+  in the request's own pages.
 """
 import itertools
 import math
@@ -501,3 +504,48 @@ def test_tree_build_chain_star_and_ties():
     assert list(tok) == [9, 0, 1, 2, 3, 2, 3, 4]
     with pytest.raises(ValueError):                         # too few candidate nodes
         tree_build(zero[:1, :1], toks[:1, :1], 9, 3)
+
+
+# ---------------------------------------------------------------- paged caches
+from oracle.cache import kv_compact_paged, kv_write_nodes_paged, paged_view  # noqa: E402
+
+
+def test_paged_view_matches_slot_loop():
+    rng = np.random.default_rng(21)
+    c = rng.integers(0, 1 << 16, size=(3, 70, 8)).astype(np.uint16)
+    r = rng.integers(0, 1 << 16, size=(3, 70, 2)).astype(np.uint16)
+    for P in (1, 8, 64):
+        cp, rp, pt = W.to_paged(c, r, P, seed=P)
+        view = paged_view(cp, pt, P)
+        for b in range(3):
+            for s_ in range(70):
+                assert (view[b, s_] == cp[pt[b, s_ // P] * P + s_ % P]).all()
+                assert (view[b, s_] == c[b, s_]).all()
+
+
+def test_paged_updates_reduce_to_contiguous_and_stay_in_their_pages():
+    rng = np.random.default_rng(22)
+    B, cap, n, P = 2, 64, 5, 16
+    c = rng.integers(0, 1 << 16, size=(B, cap, 8)).astype(np.uint16)
+    r = rng.integers(0, 1 << 16, size=(B, cap, 2)).astype(np.uint16)
+    lens = np.array([10, 40], np.int32)
+    nc = rng.integers(0, 1 << 16, size=(B, n, 8)).astype(np.uint16)
+    nr = rng.integers(0, 1 << 16, size=(B, n, 2)).astype(np.uint16)
+    path = np.array([[0, 2, 3, -1, -1], [0, 1, -1, -1, -1]], np.int32)
+    ln = np.array([3, 2], np.int32)
+    # identity table: exactly the contiguous functions
+    ident = np.arange(B * cap // P, dtype=np.int32).reshape(B, cap // P)
+    wc, wr = kv_write_nodes_paged(c.reshape(-1, 8), r.reshape(-1, 2), ident, P, lens, nc, nr)
+    ec, er = oracle.kv_write_nodes(c, r, lens, nc, nr)
+    assert (wc.reshape(B, cap, 8) == ec).all() and (wr.reshape(B, cap, 2) == er).all()
+    cc, cr, cl = kv_compact_paged(wc, wr, ident, P, lens, path, ln)
+    ec2, er2, el = oracle.kv_compact(ec, er, lens, path, ln)
+    assert (cc.reshape(B, cap, 8) == ec2).all() and (cl == el).all()
+    # shuffled pages: same logical result, spare pages untouched
+    cp, rp, pt = W.to_paged(c, r, P, seed=5, spare=4)
+    wc, wr = kv_write_nodes_paged(cp, rp, pt, P, lens, nc, nr)
+    assert (paged_view(wc, pt, P) == ec).all()
+    used = np.zeros(cp.shape[0] // P, bool)
+    used[pt.ravel()] = True
+    for q in np.nonzero(~used)[0]:
+        assert (wc[q * P:(q + 1) * P] == cp[q * P:(q + 1) * P]).all()

@@ -315,6 +315,26 @@ def draw_cache(cfg: Config, cache_lens: np.ndarray, fill: int) -> tuple[np.ndarr
     return c_kv, k_rope
 
 
+def to_paged(c_kv: np.ndarray, k_rope: np.ndarray, page_size: int, seed: int = 0, spare: int = 3):
+    """Lay per-request caches [B][cap][w] out as a shared pool of pages of page_size
+    slots, in a seeded random physical order with a few unused pages between them
+    (each request's capacity rounds up to whole pages; the extra slots are zero).
+    Returns (c_pages [N * P][512], r_pages [N * P][64], page_table int32 [B][M])."""
+    B, cap = c_kv.shape[:2]
+    M = -(-cap // page_size)
+    N = B * M + spare
+    perm = np.random.default_rng([seed, 7, page_size]).permutation(N)[: B * M].reshape(B, M)
+    c_pages = np.zeros((N * page_size, c_kv.shape[2]), dtype=c_kv.dtype)
+    r_pages = np.zeros((N * page_size, k_rope.shape[2]), dtype=k_rope.dtype)
+    for b in range(B):
+        for q in range(M):
+            lo, hi = q * page_size, min((q + 1) * page_size, cap)
+            dst = perm[b, q] * page_size
+            c_pages[dst:dst + hi - lo] = c_kv[b, lo:hi]
+            r_pages[dst:dst + hi - lo] = k_rope[b, lo:hi]
+    return c_pages, r_pages, perm.astype(np.int32)
+
+
 def draw_candidates(cfg: Config, step: int = 0, depth: int = 16, k: int = 8, vocab: int = VOCAB):
     """Drafter candidates for the tree builder: per request and depth, k distinct tokens
     with log-probabilities of a Dirichlet(1) draw, sorted from the most likely; and one
