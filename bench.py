@@ -312,6 +312,52 @@ def accept_logits_case(kd, torch, peaks, name="loop", reps=10, warm=3, requests=
             "timing": "CUDA events around each call; logits larger than L2, so no flush"}
 
 
+def paged_attn_case(kd, torch, peaks, flush, name="batched", page_size=64, reps=20, warm=3):
+    """Attention over a paged cache (the configuration's caches laid out as a shuffled
+    pool of page_size-slot pages), timed like attn_case."""
+    wl = W.make_workload(name)
+    cfg, st = wl.cfg, wl.step
+    cp, rp, pt = W.to_paged(wl.c_kv, wl.k_rope, page_size)
+    qa, qr = kd.bf16_from_bits(st.q_abs), kd.bf16_from_bits(st.q_rope)
+    gc, gr = kd.bf16_from_bits(cp), kd.bf16_from_bits(rp)
+    ptab = torch.from_numpy(pt).cuda()
+    lens = torch.from_numpy(wl.cache_lens.astype(np.int32)).cuda()
+    vis, _ = kd.kd_tree_build_mask(torch.from_numpy(st.parents).cuda())
+    ws = kd.new_workspace(cfg.B, cfg.n, cfg.H, pt.shape[1] * page_size)
+    out = torch.empty(cfg.B, cfg.n, cfg.H, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(cfg.B, cfg.n, cfg.H, dtype=torch.float32, device="cuda")
+
+    def call():
+        kd.kd_tree_verify_attn_paged(qa, qr, gc, gr, ptab, page_size, lens, vis, None, cfg.scale, out, lse, ws)
+
+    for _ in range(warm):
+        call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    times = []
+    for _ in range(reps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3)
+    del graph
+    t = float(np.median(times))
+    fl = HN.attn_flops(wl.cache_lens, [_depths(p) for p in st.parents], cfg.H)
+    res = {"workload": f"{name} over a shuffled pool of {page_size}-slot pages", "us": round(t * 1e6, 2),
+           "us_min": round(min(times) * 1e6, 2), "tflops": round(fl / t / 1e12, 1),
+           "roofline_frac": round(fl / (peaks["bf16_tflops"] * 1e12) / t, 3), "bound": "tensor",
+           "device_errors": kd.kd_read_device_error(ws),
+           "timing": "CUDA-graph replay of the call, L2 flushed (256 MB write) before each rep"}
+    del gc, gr, ws, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def tree_build_case(kd, torch, name="loop", depth=16, k=8, reps=20, warm=3):
     """Best-first draft-tree build for every request of a configuration from drafter
     candidates (depth x k per request); launch-latency sized (one warp per request)."""
@@ -457,7 +503,8 @@ def run_kd(args):
             extras = attn_extras(kd, torch, peaks, HN.L2Flush("cuda"))
             next_rows = {"accept_logits": accept_logits_case(kd, torch, peaks),
                          "causal_extend": attn_case(kd, torch, peaks, HN.L2Flush("cuda"), "extend"),
-                         "tree_build": tree_build_case(kd, torch)}
+                         "tree_build": tree_build_case(kd, torch),
+                         "paged_kv": paged_attn_case(kd, torch, peaks, HN.L2Flush("cuda"))}
         if not args.no_cpu_baseline:
             cpu = cpu_baseline(cfg, wl, host_steps[0])
 

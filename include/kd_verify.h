@@ -77,6 +77,7 @@ typedef uint16_t kd_bf16_t;
 #define KD_DEV_BAD_POSITION  0x08  /* positions[b][i] != cache_len[b] + depth(i)       */
 #define KD_DEV_TIMEOUT       0x10  /* a bounded wait inside a kernel gave up            */
 #define KD_DEV_BAD_MASK      0x20  /* a node's mask lacks bit 0 (root) or its own bit   */
+#define KD_DEV_BAD_PAGE      0x40  /* a paged cache's page id is outside the page pool  */
 
 #define KD_D_C 512
 #define KD_D_R 64
@@ -280,6 +281,53 @@ int kd_kv_write_nodes(kd_bf16_t* c_kv, kd_bf16_t* k_rope, int64_t kv_row_stride_
                       int64_t kv_row_stride_r, int64_t cap, const int32_t* cache_lens,
                       const kd_bf16_t* node_ckv, const kd_bf16_t* node_krope, int B,
                       int n, int32_t* dev_error, cudaStream_t stream);
+
+/*
+ * Paged caches.  A shared pool of pages of page_size slots replaces the per-request
+ * contiguous cache (page size 1 fragments a live service's memory: "The
+ * Architectural Keystone ...", "Assumptions Embedded in the Design").  Request b's
+ * logical slot s is row page_table[b][s / page_size] * page_size + s % page_size of
+ *   c_pages [num_pages * page_size][kv_row_stride_c] and
+ *   r_pages [num_pages * page_size][kv_row_stride_r] (bf16),
+ * page_table [B][pages_per_req] int32 (device), so a request holds
+ * cap = pages_per_req * page_size logical slots.  Pages of different requests must
+ * not overlap.  The calls below are the contiguous ones on that logical view; their
+ * results are identical to running the contiguous calls on the gathered caches.
+ */
+
+/*
+ * kd_tree_verify_attn_paged -- kd_tree_verify_attn over a paged cache.  page_size is
+ * 64, 128 or 256 and pages_per_req at most 2047; the workspace is sized by
+ * kd_verify_workspace_bytes(B, n, H, pages_per_req * page_size, kv_splits).  Page
+ * ids outside [0, num_pages) read as zero rows (no fault); KD_EINVAL otherwise as
+ * the contiguous call.
+ */
+int kd_tree_verify_attn_paged(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* q_rope,
+                              const kd_bf16_t* c_pages, const kd_bf16_t* r_pages,
+                              int64_t kv_row_stride_c, int64_t kv_row_stride_r, int page_size,
+                              const int32_t* page_table, int64_t pages_per_req, int64_t num_pages,
+                              const int32_t* cache_lens, const uint32_t* vis,
+                              const int32_t* positions, int B, int n, int H, float scale,
+                              kd_bf16_t* out, float* lse, void* workspace, size_t ws_bytes,
+                              int kv_splits, cudaStream_t stream);
+
+/*
+ * kd_kv_write_nodes_paged / kd_kv_compact_paged -- kd_kv_write_nodes and
+ * kd_kv_compact through a page table (any page_size >= 1).  A request whose slots
+ * L..L+n-1 touch a page id outside [0, num_pages) is skipped and sets
+ * KD_DEV_BAD_PAGE.  The compaction gathers rows inside the request's pages (the
+ * page table itself is not rewritten).
+ */
+int kd_kv_write_nodes_paged(kd_bf16_t* c_pages, kd_bf16_t* r_pages, int64_t kv_row_stride_c,
+                            int64_t kv_row_stride_r, int page_size, const int32_t* page_table,
+                            int64_t pages_per_req, int64_t num_pages, const int32_t* cache_lens,
+                            const kd_bf16_t* node_ckv, const kd_bf16_t* node_krope, int B, int n,
+                            int32_t* dev_error, cudaStream_t stream);
+int kd_kv_compact_paged(kd_bf16_t* c_pages, kd_bf16_t* r_pages, int64_t kv_row_stride_c,
+                        int64_t kv_row_stride_r, int page_size, const int32_t* page_table,
+                        int64_t pages_per_req, int64_t num_pages, const int32_t* path,
+                        const int32_t* len, int32_t* cache_lens, int B, int n, int32_t* dev_error,
+                        cudaStream_t stream);
 
 /*
  * kd_read_device_error -- synchronises `stream`, returns the device error word

@@ -120,7 +120,9 @@ constexpr int QK_END = K_OFF + NK * KCHUNK;
 constexpr int P_OFF = CTRL;
 constexpr int V_OFF = P_OFF + 2 * PSLOT;
 constexpr int PV_END = V_OFF + NVG * VG;
-constexpr int SMEM_BYTES = (QK_END > PV_END ? QK_END : PV_END) + 1024;
+constexpr int PT_OFF = QK_END > PV_END ? QK_END : PV_END;   // paged caches: the unit's page slice
+constexpr int PT_MAX = 2048;                                  // int32 entries (8 KB)
+constexpr int SMEM_BYTES = PT_OFF + PT_MAX * 4 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 constexpr uint32_t IDESC_QK = idesc_bf16(BM, BQ, 0, 0);    // Q, K both K-major
@@ -137,9 +139,11 @@ struct Params {
   float* part_o;
   float* part_lse;
   int32_t* err;
-  int64_t cap;
+  int64_t cap;                    // logical slots per request (pages_per_req * P when paged)
   int B, n, H, W, mtiles, splits;
   float scale_log2;
+  const int32_t* page_table;      // paged caches: [B][pages_per_req] physical page ids
+  int page_size, page_shift, pages_per_req;   // page_size = 1 << page_shift
 };
 
 struct Ctx {
@@ -209,10 +213,20 @@ __device__ __forceinline__ float max4(float a, float b, float c, float d) {
 
 // ====================================================================== QK CTA roles
 // TMA producer: Q chunks 7 and 8 once, then the K ring.
-__device__ __forceinline__ void qk_producer(const Ctx& cx, const CUtensorMap* tm_qa,
+// Cache row of request-relative key `key` of a paged cache (the unit's page-table
+// slice is in shared memory from page page0 on; keys past the last page map to row
+// 0: their scores are masked and their V rows never loaded).
+__device__ __forceinline__ int32_t paged_row(const int32_t* ptab, int page0, const Params& p, int64_t key) {
+  const int64_t pg = key >> p.page_shift;
+  return pg < p.pages_per_req ? (ptab[pg - page0] << p.page_shift) + (int32_t)(key & (p.page_size - 1)) : 0;
+}
+
+template <bool PAGED>
+__device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, const int32_t* ptab,
+                                            int page0, const CUtensorMap* tm_qa,
                                             const CUtensorMap* tm_qr, const CUtensorMap* tm_c,
                                             const CUtensorMap* tm_r, int qrow0, int64_t krow0,
-                                            int ntiles) {
+                                            int64_t kbeg, int ntiles) {
   const uint32_t base = cx.base;
   // Q: latent chunks 0..3 land in the (still unused) P staging area, chunks 4..7 in
   // K ring stages 2..3; the softmax groups move them into TMEM.  The rope chunk stays.
@@ -223,13 +237,28 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const CUtensorMap* tm
   bool ok = true;
   for (int t = 0; t < ntiles && ok; ++t) {
     const int32_t krow = (int32_t)(krow0 + (int64_t)t * BQ);
+    int32_t prow[4];                  // paged: the cache rows of the tile's (at most 4) pages
+    if (PAGED) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        prow[i] = (i << p.page_shift) < BQ ? paged_row(ptab, page0, p, kbeg + (int64_t)t * BQ + (i << p.page_shift)) : 0;
+    }
     for (int c = 0; c < NCHUNK; ++c, ++it) {
       const uint32_t st = it % NK, k = it / NK;
       if (!(ok = wait_bar(cx, cx.bar(K_EMPTY + st), (k & 1u) ^ 1u))) break;
       if (it == 2 && !(ok = wait_bar(cx, cx.bar(QT_FULL), 0))) break;   // stages 2, 3 held Q
       mbar_arrive_expect_tx(cx.bar(K_FULL + st), KCHUNK);
-      if (c < 8) tma_load_2d(base + K_OFF + st * KCHUNK, tm_c, c * KC, krow, cx.bar(K_FULL + st));
-      else tma_load_2d(base + K_OFF + st * KCHUNK, tm_r, 0, krow, cx.bar(K_FULL + st));
+      const CUtensorMap* map = c < 8 ? tm_c : tm_r;
+      const int x = c < 8 ? c * KC : 0;
+      if (!PAGED) {
+        tma_load_2d(base + K_OFF + st * KCHUNK, map, x, krow, cx.bar(K_FULL + st));
+      } else {                        // one box per page (page_size rows, 1024-byte aligned)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if ((i << p.page_shift) < BQ)
+            tma_load_2d(base + K_OFF + st * KCHUNK + (i << p.page_shift) * 128, map, x, prow[i],
+                        cx.bar(K_FULL + st));
+      }
     }
   }
   // every armed stage must have landed before the CTA may exit
@@ -453,14 +482,17 @@ __device__ __forceinline__ int group_keys(int64_t kbeg, int64_t nkeys, int t, in
   return left <= 0 ? 0 : (left < VKEYS ? (int)left : VKEYS);
 }
 
-__device__ __forceinline__ void pv_producer(const Ctx& cx, const CUtensorMap* tm_v, int64_t krow0,
+template <bool PAGED>
+__device__ __forceinline__ void pv_producer(const Ctx& cx, const Params& p, const int32_t* ptab,
+                                            int page0, const CUtensorMap* tm_v, int64_t krow0,
                                             int64_t kbeg, int64_t nkeys, int ntiles) {
   bool ok = true;
   uint32_t gi = 0;
   for (int t = 0; t < 2 * ntiles && ok; ++t) {
     for (int kh = 0; kh < BN / VKEYS && ok; ++kh) {
       if (group_keys(kbeg, nkeys, t, kh) == 0) continue;
-      const int32_t krow = (int32_t)(krow0 + (int64_t)t * BN + kh * VKEYS);
+      const int64_t key = kbeg + (int64_t)t * BN + kh * VKEYS;      // a 64-key group lies in one page
+      const int32_t krow = PAGED ? paged_row(ptab, page0, p, key) : (int32_t)(krow0 + (key - kbeg));
       for (int hh = 0; hh < 2; ++hh, ++gi) {
         const uint32_t gs = gi % NVG, k = gi / NVG;
         if (!(ok = wait_bar(cx, cx.bar(V_EMPTY + gs), (k & 1u) ^ 1u))) break;
@@ -670,6 +702,7 @@ __device__ __forceinline__ void pv_epilogue(const Ctx& cx, const Params& p, cons
 }
 
 // ====================================================================== kernel
+template <bool PAGED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant__ CUtensorMap tm_qr,
                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
@@ -752,9 +785,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + OFF_TMEM);
 
+  // paged caches: the producer warp stages the page-table slice of this unit's keys
+  const int32_t* ptab = reinterpret_cast<const int32_t*>(gbase + PT_OFF);
+  const int page0 = PAGED ? (int)(kbeg / p.page_size) : 0;
+  if (PAGED && warp == 0) {
+    const int64_t kend = kbeg + (int64_t)ntiles * BQ;
+    const int pend = (int)((kend + p.page_size - 1) / p.page_size);
+    int32_t* dst = reinterpret_cast<int32_t*>(gbase + PT_OFF);
+    for (int i = page0 + lane; i < pend && i < p.pages_per_req; i += 32)
+      dst[i - page0] = p.page_table[(size_t)b * p.pages_per_req + i];
+    __syncwarp();
+  }
+
   if (rank == 0) {
     if (warp == 0) {
-      if (lane == 0 && ntiles > 0) qk_producer(cx, &tm_qa, &tm_qr, &tm_c, &tm_r, qrow0, krow0, ntiles);
+      if (lane == 0 && ntiles > 0)
+        qk_producer<PAGED>(cx, p, ptab, page0, &tm_qa, &tm_qr, &tm_c, &tm_r, qrow0, krow0, kbeg, ntiles);
     } else if (warp == 1) {
       if (lane == 0 && ntiles > 0) qk_mma(cx, tmem, ntiles);
       __syncwarp();
@@ -763,7 +809,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
     }
   } else {
     if (warp == 0) {
-      if (lane == 0) pv_producer(cx, &tm_v, krow0, kbeg, nkeys, ntiles);
+      if (lane == 0) pv_producer<PAGED>(cx, p, ptab, page0, &tm_v, krow0, kbeg, nkeys, ntiles);
     } else if (warp == 1) {
       pv_mma(cx, gbase, tmem, kbeg, nkeys, ntiles);
     } else {
@@ -869,7 +915,7 @@ static int active_pairs(int sms) {
   cfg.attrs = &at;
   cfg.numAttrs = 1;
   int nc = 0;
-  if (cudaOccupancyMaxActiveClusters(&nc, attn_tc_kernel, &cfg) == cudaSuccess && nc > 0) pairs = nc;
+  if (cudaOccupancyMaxActiveClusters(&nc, attn_tc_kernel<false>, &cfg) == cudaSuccess && nc > 0) pairs = nc;
   cudaGetLastError();
   if (dev >= 0 && dev < 64) cached[dev] = pairs;
   return pairs;
@@ -914,12 +960,16 @@ extern "C" size_t kd_verify_workspace_bytes(int B, int n, int H, int64_t cap, in
   return workspace_bytes_for(B, n, H, s);
 }
 
-extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_rope,
-                                   const kd_bf16_t* c_kv, const kd_bf16_t* k_rope, int64_t sc,
-                                   int64_t sr, int64_t cap, const int32_t* cache_lens,
-                                   const uint32_t* vis, const int32_t* positions, int B, int n,
-                                   int H, float scale, kd_bf16_t* out, float* lse, void* workspace,
-                                   size_t ws_bytes, int kv_splits, cudaStream_t stream) {
+// Both entry points: a contiguous cache (page_table == nullptr; cache rows B * cap) or a
+// paged one (cache rows num_pages * page_size, cap = pages_per_req * page_size).
+static int verify_attn_impl(const kd_bf16_t* q_abs, const kd_bf16_t* q_rope, const kd_bf16_t* c_kv,
+                            const kd_bf16_t* k_rope, int64_t sc, int64_t sr, int64_t cap,
+                            const int32_t* cache_lens, const uint32_t* vis, const int32_t* positions,
+                            int B, int n, int H, float scale, kd_bf16_t* out, float* lse,
+                            void* workspace, size_t ws_bytes, int kv_splits, const int32_t* page_table,
+                            int page_size, int64_t pages_per_req, int64_t num_pages,
+                            cudaStream_t stream) {
+  const bool paged = page_table != nullptr;
   if (!q_abs || !q_rope || !cache_lens || !vis || !out || !lse || !workspace ||
       !shapes_ok(B, n) || H < 1 || H > KD_MAX_HEADS || !cache_ok(c_kv, k_rope, sc, sr, cap) ||
       !aligned16(q_abs) || !aligned16(q_rope) || !aligned16(out) ||
@@ -927,7 +977,8 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
       kv_splits > 64)
     return KD_EINVAL;
   const int64_t rows = (int64_t)B * n * H;
-  if (rows > INT32_MAX || (int64_t)B * cap > INT32_MAX) return KD_EINVAL;
+  const int64_t cache_rows = paged ? num_pages * page_size : (int64_t)B * cap;
+  if (rows > INT32_MAX || cache_rows > INT32_MAX) return KD_EINVAL;
   int sms = 0;
   int st = device_sms(&sms);
   if (st) return st;
@@ -935,9 +986,13 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    st = cuda_status(cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          tc::SMEM_BYTES),
+    st = cuda_status(cudaFuncSetAttribute(tc::attn_tc_kernel<false>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES),
                      "cudaFuncSetAttribute(attn_tc_kernel)");
+    if (st) return st;
+    st = cuda_status(cudaFuncSetAttribute(tc::attn_tc_kernel<true>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES),
+                     "cudaFuncSetAttribute(attn_tc_kernel, paged)");
     if (st) return st;
     attr_set[dev] = true;
   }
@@ -951,9 +1006,10 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   CUtensorMap tq, tr, tcv, tkr, tv, to, tpo;
   if ((st = tc::make_map(&tq, q_abs, KD_D_C, (uint64_t)rows, KD_D_C * 2, tc::BM))) return st;
   if ((st = tc::make_map(&tr, q_rope, KD_D_R, (uint64_t)rows, KD_D_R * 2, tc::BM))) return st;
-  if ((st = tc::make_map(&tcv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::BQ))) return st;
-  if ((st = tc::make_map(&tkr, k_rope, KD_D_R, (uint64_t)(B * cap), (uint64_t)sr * 2, tc::BQ))) return st;
-  if ((st = tc::make_map(&tv, c_kv, KD_D_C, (uint64_t)(B * cap), (uint64_t)sc * 2, tc::VKEYS))) return st;
+  const uint32_t kbox = paged ? (uint32_t)page_size : (uint32_t)tc::BQ;    // K box rows (one page)
+  if ((st = tc::make_map(&tcv, c_kv, KD_D_C, (uint64_t)cache_rows, (uint64_t)sc * 2, kbox))) return st;
+  if ((st = tc::make_map(&tkr, k_rope, KD_D_R, (uint64_t)cache_rows, (uint64_t)sr * 2, kbox))) return st;
+  if ((st = tc::make_map(&tv, c_kv, KD_D_C, (uint64_t)cache_rows, (uint64_t)sc * 2, tc::VKEYS))) return st;
   if ((st = tc::make_out_map(&to, out, (uint64_t)rows / B, (uint64_t)B))) return st;
 
   tc::Params prm;
@@ -975,6 +1031,10 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   prm.mtiles = (int)((rows / B + tc::BM - 1) / tc::BM);
   prm.splits = splits;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.page_table = page_table;
+  prm.page_size = paged ? page_size : 1;
+  prm.page_shift = paged ? (page_size == 64 ? 6 : page_size == 128 ? 7 : 8) : 0;
+  prm.pages_per_req = paged ? (int)pages_per_req : 0;
   if (splits > 1) {
     if ((st = tc::make_part_map(&tpo, prm.part_o, (uint64_t)rows / B, (uint64_t)splits * B))) return st;
   } else {
@@ -982,11 +1042,42 @@ extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_ro
   }
   const int64_t units = (int64_t)B * prm.mtiles * splits;
   if (2 * units > INT32_MAX) return KD_EINVAL;
-  tc::attn_tc_kernel<<<dim3((unsigned)(2 * units)), tc::NTHREADS, tc::SMEM_BYTES, stream>>>(
-      tq, tr, tcv, tkr, tv, to, tpo, prm);
+  if (paged)
+    tc::attn_tc_kernel<true><<<dim3((unsigned)(2 * units)), tc::NTHREADS, tc::SMEM_BYTES, stream>>>(
+        tq, tr, tcv, tkr, tv, to, tpo, prm);
+  else
+    tc::attn_tc_kernel<false><<<dim3((unsigned)(2 * units)), tc::NTHREADS, tc::SMEM_BYTES, stream>>>(
+        tq, tr, tcv, tkr, tv, to, tpo, prm);
   st = launch_status("attn_tc_kernel");
   if (st || splits == 1) return st;
   return launch_combine(prm.part_o, prm.part_lse, cache_lens, B, n, H, cap, splits, out, lse, stream);
+}
+
+extern "C" int kd_tree_verify_attn(const kd_bf16_t* q_abs, const kd_bf16_t* q_rope,
+                                   const kd_bf16_t* c_kv, const kd_bf16_t* k_rope, int64_t sc,
+                                   int64_t sr, int64_t cap, const int32_t* cache_lens,
+                                   const uint32_t* vis, const int32_t* positions, int B, int n,
+                                   int H, float scale, kd_bf16_t* out, float* lse, void* workspace,
+                                   size_t ws_bytes, int kv_splits, cudaStream_t stream) {
+  return verify_attn_impl(q_abs, q_rope, c_kv, k_rope, sc, sr, cap, cache_lens, vis, positions, B, n,
+                          H, scale, out, lse, workspace, ws_bytes, kv_splits, nullptr, 1, 0, 0, stream);
+}
+
+extern "C" int kd_tree_verify_attn_paged(const kd_bf16_t* q_abs, const kd_bf16_t* q_rope,
+                                         const kd_bf16_t* c_pages, const kd_bf16_t* r_pages,
+                                         int64_t sc, int64_t sr, int page_size,
+                                         const int32_t* page_table, int64_t pages_per_req,
+                                         int64_t num_pages, const int32_t* cache_lens,
+                                         const uint32_t* vis, const int32_t* positions, int B, int n,
+                                         int H, float scale, kd_bf16_t* out, float* lse,
+                                         void* workspace, size_t ws_bytes, int kv_splits,
+                                         cudaStream_t stream) {
+  if (!page_table || (page_size != 64 && page_size != 128 && page_size != 256) || pages_per_req < 1 ||
+      pages_per_req + 1 > tc::PT_MAX || num_pages < 1)
+    return KD_EINVAL;
+  return verify_attn_impl(q_abs, q_rope, c_pages, r_pages, sc, sr, pages_per_req * page_size,
+                          cache_lens, vis, positions, B, n, H, scale, out, lse, workspace, ws_bytes,
+                          kv_splits, page_table, page_size, pages_per_req, num_pages, stream);
 }
 
 // ================================================================== allocation-free variant

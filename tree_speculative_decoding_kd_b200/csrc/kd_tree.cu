@@ -94,27 +94,55 @@ accept_kernel(const int32_t* __restrict__ tokens, const int32_t* __restrict__ pa
   accept_walk(tokens, parents, argmax, b, n, path, len, bonus, dev_error);
 }
 
+// ------------------------------------------------------------------ slot -> cache row
+// A request's logical slot s lives in cache row b * cap + s (contiguous caches) or in
+// row page_table[b][s / P] * P + s % P of a shared page pool (paged caches: page size
+// P > 1, the remedy for the page-size-1 fragmentation of "The Architectural Keystone",
+// "Assumptions Embedded in the Design").
+struct SlotMap {
+  const int32_t* pt;          // [B][M] physical page ids, or nullptr for a contiguous cache
+  int64_t cap;                // logical slots per request
+  int64_t pages;              // pages in the pool (paged)
+  int P, M;                   // page size, pages per request (paged)
+  __device__ int64_t row(int b, int64_t s) const {
+    return pt ? (int64_t)pt[(size_t)b * M + s / P] * P + s % P : (int64_t)b * cap + s;
+  }
+  // every page holding slots [s0, s1) is inside the pool (always true when contiguous)
+  __device__ bool pages_ok(int b, int64_t s0, int64_t s1) const {
+    if (!pt) return true;
+    for (int64_t q = s0 / P; q <= (s1 - 1) / P; ++q) {
+      const int32_t v = pt[(size_t)b * M + q];
+      if (v < 0 || v >= pages) return false;
+    }
+    return true;
+  }
+};
+
 // ------------------------------------------------------------------ node write
 // One CTA per request; 16-byte copies of the n node rows into slots L..L+n-1.
 __global__ void __launch_bounds__(256)
 write_nodes_kernel(uint4* __restrict__ c_kv, uint4* __restrict__ k_rope, int64_t sc16,
-                   int64_t sr16, int64_t cap, const int32_t* __restrict__ cache_lens,
+                   int64_t sr16, SlotMap map, const int32_t* __restrict__ cache_lens,
                    const uint4* __restrict__ node_ckv, const uint4* __restrict__ node_krope,
                    int n, int32_t* dev_error) {
   const int b = blockIdx.x;
   const int64_t L = cache_lens[b];
-  if (L < 0 || L + n > cap) {
+  if (L < 0 || L + n > map.cap) {
     if (threadIdx.x == 0) raise_dev_error(dev_error, KD_DEV_CACHE_FULL);
     return;
   }
+  if (!map.pages_ok(b, L, L + n)) {
+    if (threadIdx.x == 0) raise_dev_error(dev_error, KD_DEV_BAD_PAGE);
+    return;
+  }
   constexpr int CC = KD_D_C / 8, CR = KD_D_R / 8;   // uint4 per row
-  const int64_t row0 = (int64_t)b * cap + L;
   for (int idx = threadIdx.x; idx < n * (CC + CR); idx += blockDim.x) {
     const int k = idx / (CC + CR), q = idx % (CC + CR);
+    const int64_t r = map.row(b, L + k);
     if (q < CC)
-      c_kv[(row0 + k) * sc16 + q] = node_ckv[((size_t)b * n + k) * CC + q];
+      c_kv[r * sc16 + q] = node_ckv[((size_t)b * n + k) * CC + q];
     else
-      k_rope[(row0 + k) * sr16 + (q - CC)] = node_krope[((size_t)b * n + k) * CR + (q - CC)];
+      k_rope[r * sr16 + (q - CC)] = node_krope[((size_t)b * n + k) * CR + (q - CC)];
   }
 }
 
@@ -124,7 +152,7 @@ write_nodes_kernel(uint4* __restrict__ c_kv, uint4* __restrict__ k_rope, int64_t
 // already in place.  Shared memory holds up to n rows of 1152 bytes.
 __global__ void __launch_bounds__(256)
 compact_kernel(uint4* __restrict__ c_kv, uint4* __restrict__ k_rope, int64_t sc16, int64_t sr16,
-               int64_t cap, const int32_t* __restrict__ path, const int32_t* __restrict__ len,
+               SlotMap map, const int32_t* __restrict__ path, const int32_t* __restrict__ len,
                int32_t* __restrict__ cache_lens, int n, int32_t* dev_error) {
   extern __shared__ uint4 stage[];
   __shared__ int src[KD_MAX_NODES], dst[KD_MAX_NODES];
@@ -136,7 +164,8 @@ compact_kernel(uint4* __restrict__ c_kv, uint4* __restrict__ k_rope, int64_t sc1
   if (threadIdx.x == 0) {
     int good = 1, err = 0;
     if (m < 1 || m > n) { good = 0; err |= KD_DEV_BAD_PATH; }
-    if (L < 0 || L + n > cap) { good = 0; err |= KD_DEV_CACHE_FULL; }
+    if (L < 0 || L + n > map.cap) { good = 0; err |= KD_DEV_CACHE_FULL; }
+    else if (!map.pages_ok(b, L, L + n)) { good = 0; err |= KD_DEV_BAD_PAGE; }
     int c = 0;
     for (int j = 0; good && j < m; ++j) {
       const int p = path[(size_t)b * n + j];
@@ -149,17 +178,16 @@ compact_kernel(uint4* __restrict__ c_kv, uint4* __restrict__ k_rope, int64_t sc1
   }
   __syncthreads();
   if (!ok) return;
-  const int64_t row0 = (int64_t)b * cap + L;
   const int total = moves * ROW;
   for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {      // read all ...
     const int r = idx / ROW, q = idx % ROW;
-    const int64_t s = row0 + src[r];
+    const int64_t s = map.row(b, L + src[r]);
     stage[idx] = (q < CC) ? c_kv[s * sc16 + q] : k_rope[s * sr16 + (q - CC)];
   }
   __syncthreads();
   for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {      // ... then write
     const int r = idx / ROW, q = idx % ROW;
-    const int64_t d = row0 + dst[r];
+    const int64_t d = map.row(b, L + dst[r]);
     if (q < CC) c_kv[d * sc16 + q] = stage[idx];
     else k_rope[d * sr16 + (q - CC)] = stage[idx];
   }
@@ -203,22 +231,42 @@ extern "C" int kd_kv_write_nodes(kd_bf16_t* c_kv, kd_bf16_t* k_rope, int64_t sc,
     return KD_EINVAL;
   int st = device_sms(nullptr);
   if (st) return st;
+  const SlotMap map{nullptr, cap, 0, 1, 0};
   write_nodes_kernel<<<B, 256, 0, stream>>>(
-      reinterpret_cast<uint4*>(c_kv), reinterpret_cast<uint4*>(k_rope), sc / 8, sr / 8, cap,
+      reinterpret_cast<uint4*>(c_kv), reinterpret_cast<uint4*>(k_rope), sc / 8, sr / 8, map,
       cache_lens, reinterpret_cast<const uint4*>(node_ckv),
       reinterpret_cast<const uint4*>(node_krope), n, dev_error);
   return launch_status("write_nodes_kernel");
 }
 
-extern "C" int kd_kv_compact(kd_bf16_t* c_kv, kd_bf16_t* k_rope, int64_t sc, int64_t sr,
-                             int64_t cap, const int32_t* path, const int32_t* len,
-                             int32_t* cache_lens, int B, int n, int32_t* dev_error,
-                             cudaStream_t stream) {
-  if (!cache_ok(c_kv, k_rope, sc, sr, cap) || !path || !len || !cache_lens || !shapes_ok(B, n))
+static bool paged_ok(const int32_t* page_table, int page_size, int64_t pages_per_req, int64_t num_pages) {
+  return page_table && page_size >= 1 && pages_per_req >= 1 && num_pages >= 1 &&
+         num_pages * page_size <= (int64_t)INT32_MAX && pages_per_req * page_size <= (int64_t)INT32_MAX;
+}
+
+extern "C" int kd_kv_write_nodes_paged(kd_bf16_t* c_pages, kd_bf16_t* r_pages, int64_t sc, int64_t sr,
+                                       int page_size, const int32_t* page_table, int64_t pages_per_req,
+                                       int64_t num_pages, const int32_t* cache_lens,
+                                       const kd_bf16_t* node_ckv, const kd_bf16_t* node_krope, int B,
+                                       int n, int32_t* dev_error, cudaStream_t stream) {
+  if (!paged_ok(page_table, page_size, pages_per_req, num_pages) ||
+      !cache_ok(c_pages, r_pages, sc, sr, num_pages * page_size) || !cache_lens || !node_ckv ||
+      !node_krope || !aligned16(node_ckv) || !aligned16(node_krope) || !shapes_ok(B, n))
     return KD_EINVAL;
   int st = device_sms(nullptr);
   if (st) return st;
-  const size_t smem = (size_t)n * (KD_D_C + KD_D_R) * 2;
+  const SlotMap map{page_table, pages_per_req * page_size, num_pages, page_size, (int)pages_per_req};
+  write_nodes_kernel<<<B, 256, 0, stream>>>(
+      reinterpret_cast<uint4*>(c_pages), reinterpret_cast<uint4*>(r_pages), sc / 8, sr / 8, map,
+      cache_lens, reinterpret_cast<const uint4*>(node_ckv),
+      reinterpret_cast<const uint4*>(node_krope), n, dev_error);
+  return launch_status("write_nodes_kernel");
+}
+
+// Device check plus the compaction kernel's shared-memory limit (once per device).
+static int compact_setup() {
+  int st = device_sms(nullptr);
+  if (st) return st;
   static bool attr_set[64];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -229,8 +277,40 @@ extern "C" int kd_kv_compact(kd_bf16_t* c_kv, kd_bf16_t* k_rope, int64_t sc, int
     if (st) return st;
     attr_set[dev] = true;
   }
+  return KD_OK;
+}
+
+extern "C" int kd_kv_compact(kd_bf16_t* c_kv, kd_bf16_t* k_rope, int64_t sc, int64_t sr,
+                             int64_t cap, const int32_t* path, const int32_t* len,
+                             int32_t* cache_lens, int B, int n, int32_t* dev_error,
+                             cudaStream_t stream) {
+  if (!cache_ok(c_kv, k_rope, sc, sr, cap) || !path || !len || !cache_lens || !shapes_ok(B, n))
+    return KD_EINVAL;
+  int st = compact_setup();
+  if (st) return st;
+  const size_t smem = (size_t)n * (KD_D_C + KD_D_R) * 2;
+  const SlotMap map{nullptr, cap, 0, 1, 0};
   compact_kernel<<<B, 256, smem, stream>>>(reinterpret_cast<uint4*>(c_kv),
-                                           reinterpret_cast<uint4*>(k_rope), sc / 8, sr / 8, cap,
+                                           reinterpret_cast<uint4*>(k_rope), sc / 8, sr / 8, map,
+                                           path, len, cache_lens, n, dev_error);
+  return launch_status("compact_kernel");
+}
+
+extern "C" int kd_kv_compact_paged(kd_bf16_t* c_pages, kd_bf16_t* r_pages, int64_t sc, int64_t sr,
+                                   int page_size, const int32_t* page_table, int64_t pages_per_req,
+                                   int64_t num_pages, const int32_t* path, const int32_t* len,
+                                   int32_t* cache_lens, int B, int n, int32_t* dev_error,
+                                   cudaStream_t stream) {
+  if (!paged_ok(page_table, page_size, pages_per_req, num_pages) ||
+      !cache_ok(c_pages, r_pages, sc, sr, num_pages * page_size) || !path || !len || !cache_lens ||
+      !shapes_ok(B, n))
+    return KD_EINVAL;
+  int st = compact_setup();
+  if (st) return st;
+  const size_t smem = (size_t)n * (KD_D_C + KD_D_R) * 2;
+  const SlotMap map{page_table, pages_per_req * page_size, num_pages, page_size, (int)pages_per_req};
+  compact_kernel<<<B, 256, smem, stream>>>(reinterpret_cast<uint4*>(c_pages),
+                                           reinterpret_cast<uint4*>(r_pages), sc / 8, sr / 8, map,
                                            path, len, cache_lens, n, dev_error);
   return launch_status("compact_kernel");
 }

@@ -39,6 +39,11 @@ _SIGS = {
     "kd_tree_accept": (_i, [_p, _p, _p, _i, _i, _p, _p, _p, _p, _p]),
     "kd_accept_workspace_bytes": (_sz, [_i, _i]),
     "kd_tree_build": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p]),
+    "kd_tree_verify_attn_paged": (_i, [_p, _p, _p, _p, _i64, _i64, _i, _p, _i64, _i64, _p, _p, _p, _i,
+                                       _i, _i, _f, _p, _p, _p, _sz, _i, _p]),
+    "kd_kv_write_nodes_paged": (_i, [_p, _p, _i64, _i64, _i, _p, _i64, _i64, _p, _p, _p, _i, _i, _p,
+                                     _p]),
+    "kd_kv_compact_paged": (_i, [_p, _p, _i64, _i64, _i, _p, _i64, _i64, _p, _p, _p, _i, _i, _p, _p]),
     "kd_tree_accept_logits": (_i, [_p, _p, _p, _i, _i, _i64, _p, _p, _p, _p, _p, _sz, _p, _p]),
     "kd_kv_compact": (_i, [_p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _p, _p]),
     "kd_kv_write_nodes": (_i, [_p, _p, _i64, _i64, _i64, _p, _p, _p, _i, _i, _p, _p]),
@@ -52,7 +57,7 @@ for _name, (_res, _args) in _SIGS.items():
 
 D_C, D_R = 512, 64
 KD_DEV_BITS = {0x01: "BAD_PARENT", 0x02: "CACHE_FULL", 0x04: "BAD_PATH",
-               0x08: "BAD_POSITION", 0x10: "TIMEOUT", 0x20: "BAD_MASK"}
+               0x08: "BAD_POSITION", 0x10: "TIMEOUT", 0x20: "BAD_MASK", 0x40: "BAD_PAGE"}
 
 
 class KdError(RuntimeError):
@@ -274,6 +279,72 @@ def kd_kv_write_nodes(c_kv, k_rope, cache_lens, node_ckv, node_krope, dev_error=
     _check(lib.kd_kv_write_nodes(_ptr(c_kv), _ptr(k_rope), sc, sr, cap, _ptr(cache_lens),
                                  _ptr(node_ckv), _ptr(node_krope), B, n, _ptr(dev_error),
                                  _stream(stream)), "kd_kv_write_nodes")
+
+
+def _page_args(c_pages, r_pages, page_table, page_size):
+    """Strides, pages per request and pool size of a paged cache: pools [rows][512] /
+    [rows][64] bf16 (rows = num_pages * page_size), page_table int32 [B][M]."""
+    _need(c_pages, torch.bfloat16, "c_pages", contiguous=False)
+    _need(r_pages, torch.bfloat16, "r_pages", contiguous=False)
+    _need(page_table, torch.int32, "page_table")
+    rows = c_pages.shape[0]
+    if c_pages.dim() != 2 or c_pages.shape[1] != D_C or tuple(r_pages.shape) != (rows, D_R):
+        raise ValueError("c_pages must be [rows][512] and r_pages [rows][64]")
+    if rows % page_size:
+        raise ValueError("pool rows must be a multiple of page_size")
+    for t in (c_pages, r_pages):
+        if t.stride(1) != 1:
+            raise ValueError("pool rows must be unit-stride")
+    return c_pages.stride(0), r_pages.stride(0), page_table.shape[1], rows // page_size
+
+
+def kd_tree_verify_attn_paged(q_abs, q_rope, c_pages, r_pages, page_table, page_size, cache_lens, vis,
+                              positions=None, scale=1.0 / math.sqrt(192.0), out=None, lse=None,
+                              workspace=None, kv_splits=0, stream=None):
+    sc, sr, M, N = _page_args(c_pages, r_pages, page_table, page_size)
+    _need(q_abs, torch.bfloat16, "q_abs")
+    _need(q_rope, torch.bfloat16, "q_rope")
+    _need(cache_lens, torch.int32, "cache_lens")
+    _need(vis, (torch.int32, torch.uint32), "vis")
+    B, n, H, _ = q_abs.shape
+    if positions is not None:
+        _need(positions, torch.int32, "positions")
+    out = torch.empty(B, n, H, D_C, dtype=torch.bfloat16, device=q_abs.device) if out is None else out
+    lse = torch.empty(B, n, H, dtype=torch.float32, device=q_abs.device) if lse is None else lse
+    if workspace is None:
+        workspace = new_workspace(B, n, H, M * page_size, kv_splits, q_abs.device)
+    _check(lib.kd_tree_verify_attn_paged(_ptr(q_abs), _ptr(q_rope), _ptr(c_pages), _ptr(r_pages), sc, sr,
+                                         int(page_size), _ptr(page_table), M, N, _ptr(cache_lens),
+                                         _ptr(vis), _ptr(positions), B, n, H, float(scale), _ptr(out),
+                                         _ptr(lse), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), int(kv_splits),
+                                         _stream(stream)), "kd_tree_verify_attn_paged")
+    return out, lse
+
+
+def kd_kv_write_nodes_paged(c_pages, r_pages, page_table, page_size, cache_lens, node_ckv, node_krope,
+                            dev_error=None, stream=None):
+    sc, sr, M, N = _page_args(c_pages, r_pages, page_table, page_size)
+    _need(node_ckv, torch.bfloat16, "node_ckv")
+    _need(node_krope, torch.bfloat16, "node_krope")
+    _need(cache_lens, torch.int32, "cache_lens")
+    B, n, _ = node_ckv.shape
+    _check(lib.kd_kv_write_nodes_paged(_ptr(c_pages), _ptr(r_pages), sc, sr, int(page_size),
+                                       _ptr(page_table), M, N, _ptr(cache_lens), _ptr(node_ckv),
+                                       _ptr(node_krope), B, n, _ptr(dev_error), _stream(stream)),
+           "kd_kv_write_nodes_paged")
+
+
+def kd_kv_compact_paged(c_pages, r_pages, page_table, page_size, path, length, cache_lens, dev_error=None,
+                        stream=None):
+    sc, sr, M, N = _page_args(c_pages, r_pages, page_table, page_size)
+    _need(path, torch.int32, "path")
+    _need(length, torch.int32, "len")
+    _need(cache_lens, torch.int32, "cache_lens")
+    B, n = path.shape
+    _check(lib.kd_kv_compact_paged(_ptr(c_pages), _ptr(r_pages), sc, sr, int(page_size), _ptr(page_table),
+                                   M, N, _ptr(path), _ptr(length), _ptr(cache_lens), B, n,
+                                   _ptr(dev_error), _stream(stream)), "kd_kv_compact_paged")
 
 
 def kd_read_device_error(word, clear=True, stream=None) -> int:
