@@ -81,3 +81,44 @@ def test_host_validation_rejects_before_cuda(lib):
     bad = list(args); bad[18] = 65                   # too many splits
     assert lib.kd_tree_verify_attn(*bad) == -1
     assert lib.kd_read_device_error(None, 0, None) == -1
+
+
+def test_host_validation_of_the_widened_calls(lib):
+    """Fused argmax + accept, tree build and paged caches reject bad arguments on the
+    host (KD_EINVAL = -1, KD_ERANGE = -2) without a device."""
+    from tree_speculative_decoding_kd_b200 import kd
+    V = ctypes.c_void_p
+    # accept workspace: 8 B ranks per node, 4 B counters per request (16-byte aligned), tokens
+    assert kd.lib.kd_accept_workspace_bytes(2, 17) == 288 + 2 * 17 * 4
+    assert kd.lib.kd_accept_workspace_bytes(0, 17) == 0 and kd.lib.kd_accept_workspace_bytes(1, 129) == 0
+    ok = [V(16), V(16), V(16), 2, 17, 163840, None, V(16), V(16), V(16), V(256), 4096, None, None]
+    bad = list(ok); bad[5] = 163842                  # vocabulary not a multiple of 4
+    assert lib.kd_tree_accept_logits(*bad) == -1
+    bad = list(ok); bad[2] = V(24)                   # logits not 16-byte aligned
+    assert lib.kd_tree_accept_logits(*bad) == -1
+    bad = list(ok); bad[10] = None                   # no workspace
+    assert lib.kd_tree_accept_logits(*bad) == -1
+    bad = list(ok); bad[11] = 100                    # workspace too small
+    assert lib.kd_tree_accept_logits(*bad) == -2
+    # tree build: shapes, and enough candidate nodes for n
+    tb = [V(16), V(16), V(16), 2, 16, 8, 17, V(16), V(16), None, None, None]
+    for i, v in ((5, 0), (5, 256), (6, 129), (4, 0), (0, None)):
+        bad = list(tb); bad[i] = v
+        assert lib.kd_tree_build(*bad) == -1
+    bad = list(tb); bad[4], bad[5], bad[6] = 1, 2, 4  # 2 candidate nodes, 3 needed
+    assert lib.kd_tree_build(*bad) == -1
+    # paged attention: page size, page table, slice limit
+    pa = [V(16), V(16), V(16), V(16), 512, 64, 64, V(16), 100, 1000, V(16), V(16), None, 1, 8, 16, 0.1,
+          V(16), V(16), V(256), 1 << 20, 0, None]
+    for i, v in ((6, 100), (7, None), (8, 2048), (9, 0)):
+        bad = list(pa); bad[i] = v
+        assert lib.kd_tree_verify_attn_paged(*bad) == -1
+    # paged node write / compaction
+    pw = [V(16), V(16), 512, 64, 16, V(16), 10, 100, V(16), V(16), V(16), 1, 8, None, None]
+    for i, v in ((5, None), (4, 0), (7, 0)):
+        bad = list(pw); bad[i] = v
+        assert lib.kd_kv_write_nodes_paged(*bad) == -1
+    pc = [V(16), V(16), 512, 64, 16, V(16), 10, 100, V(16), V(16), V(16), 1, 8, None, None]
+    for i, v in ((5, None), (4, 0), (6, 0)):
+        bad = list(pc); bad[i] = v
+        assert lib.kd_kv_compact_paged(*bad) == -1
