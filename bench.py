@@ -33,17 +33,26 @@ METRIC = "tree-verify MLA attn TFLOP/s + KV HBM GB/s (% roofline); verify steps/
 N_DISTINCT = 8          # distinct pre-generated step inputs, cycled
 
 
+def code_sha256_16(path):
+    """sha256 (first 16 hex digits) of a CUDA source with its comments and whitespace
+    removed, so that it changes exactly when the code does."""
+    import hashlib
+    import re
+    src = open(path).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return hashlib.sha256("".join(src.split()).encode()).hexdigest()[:16]
+
+
 def profiled_traffic():
     """DRAM bytes per attention launch from the committed ncu summary, only while the
-    attention kernel source is the one those counters were taken from (else None)."""
-    import hashlib
+    attention kernel's code is the one those counters were taken from (else None)."""
     prof = os.path.join(ROOT, "profiles", "verify_step_loop_launch_list.md")
     src = os.path.join(ROOT, "tree_speculative_decoding_kd_b200", "csrc", "kd_attn_tc.cu")
     try:
         text = open(prof).read()
-        want = text.split("kernel_source_sha256_16:")[1].split()[0]
-        have = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if want != have:
+        want = text.split("kernel_code_sha256_16:")[1].split()[0]
+        if want != code_sha256_16(src):
             return None
         return int(text.split("traffic_bytes_per_launch:")[1].split()[0])
     except (OSError, IndexError, ValueError):

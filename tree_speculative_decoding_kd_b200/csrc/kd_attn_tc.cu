@@ -11,11 +11,12 @@
 // Because the latent is shared by all heads, a request's n*H query rows against
 // its keys form a dense (n*H x 576) . (576 x keys) contraction followed by a
 // (n*H x keys) . (keys x 512) one.  Rows are node-major (row = i*H + h) and cut
-// into 128-row M tiles; keys are streamed in 128-key tiles.
+// into 128-row M tiles; keys are streamed in 256-key QK tiles, each split into two
+// 128-key P tiles.
 //
 // The fp32 output accumulator of one M tile (128 x 512) fills all 512 TMEM
-// columns of an SM, leaving none for scores, so each unit of work runs on a
-// 2-CTA cluster with split roles:
+// columns of an SM, leaving none for scores, so each unit of work (request, M tile,
+// key partition) runs on a 2-CTA cluster with split roles:
 //   rank 0 ("QK" CTA): S = Q K^T for 256 keys at a time (M=128, N=256 MMAs, the
 //       shape that keeps the tensor pipe saturated from one issuing thread) into
 //       256 TMEM columns.  The eight 64-wide latent chunks of Q sit in the other 256
@@ -23,17 +24,26 @@
 //       chunk sits in shared memory.  Shared memory holds a 4-stage ring of
 //       256-key x 64-column K chunks (TMA, 128-byte swizzle) and two P staging
 //       slots.  Two 4-warp softmax groups copy S into registers (freeing TMEM for
-//       the next tile at once), keep an online max with a lazy rescale threshold,
-//       and emit P as two 128-key halves: each is written into a local staging slot
-//       in the K-major swizzled layout the MMA reads and moved to rank 1 by one
-//       thread with a single bulk copy that completes on rank 1's barrier.
+//       the next tile at once), take the row max on raw scores with the
+//       three-operand max, keep an online max with a lazy rescale threshold, and
+//       emit P as two 128-key halves (scale and reference folded into one packed
+//       f32x2 FMA per key pair, sums in packed f32x2 adds): each half is written
+//       into a local staging slot in the K-major swizzled layout the MMA reads and
+//       moved to rank 1 by one thread with a single bulk copy that completes on
+//       rank 1's barrier.
 //   rank 1 ("PV" CTA): O (128 x 512 fp32) in TMEM; V as 64-key x 256-column
 //       groups (four 64-column MN-major boxes) in a 4-deep ring; O += P V as
-//       M=128, N=256, K=16 MMAs; two 4-warp groups apply the rare O rescale and
-//       write the normalised output (or a split-KV partial), 256 columns each.
+//       M=128, N=256, K=16 MMAs; V groups wholly past the request's last key are
+//       neither loaded nor multiplied.  Two 4-warp groups apply the rare O rescale
+//       and write the normalised bf16 output (or an fp32 split-KV partial) through
+//       swizzled shared-memory boxes and TMA stores, 256 columns each.
 // QK work (576-deep) and PV work (512-deep) are nearly equal, so the pair keeps
 // both tensor pipes busy.  Both CTAs read the same c_kv tile (the second read
-// hits L2).  No TMA multicast is used anywhere.
+// hits L2).  Units go out longest request first.  No TMA multicast is used anywhere.
+//
+// attn_tc_kernel<true> reads a paged cache instead: each 256-key K stage arrives as
+// one TMA box per page and each 64-key V group as one box inside a page, from the
+// unit's slice of the page table staged in shared memory; nothing else differs.
 //
 // Every mbarrier wait is bounded (globaltimer); a wait that gives up raises
 // KD_DEV_TIMEOUT, marks both CTAs aborted, and every role falls through to the
