@@ -474,33 +474,51 @@ def run_kd(args):
     pinned = []
     for ds in dsteps:
         pinned.append([t.cpu().pin_memory() for t in ds.tensors()])
-    stage = DeviceStep.__new__(DeviceStep)
-    stage.q_abs, stage.q_rope, stage.node_ckv, stage.node_krope, stage.parents, stage.tokens, \
-        stage.argmax = [t.clone() for t in dsteps[0].tensors()]
+    # two device stages: step s+1's inputs upload on a copy stream while step s computes
+    stages = [DeviceStep.__new__(DeviceStep) for _ in range(2)]
+    for sg in stages:
+        sg.q_abs, sg.q_rope, sg.node_ckv, sg.node_krope, sg.parents, sg.tokens, \
+            sg.argmax = [t.clone() for t in dsteps[0].tensors()]
     res_host = [torch.empty(cfg.B, cfg.n, dtype=torch.int32).pin_memory(),
                 torch.empty(cfg.B, dtype=torch.int32).pin_memory(),
                 torch.empty(cfg.B, dtype=torch.int32).pin_memory()]
     h2d = sum(t.numel() * t.element_size() for t in pinned[0])
     d2h = sum(t.numel() * t.element_size() for t in res_host)
+    comp, copy_s = torch.cuda.current_stream(), torch.cuda.Stream()
+    ready = [torch.cuda.Event() for _ in range(2)]
+    free = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step(s):
-        for dst, src in zip(stage.tensors(), pinned[s % N_DISTINCT]):
-            dst.copy_(src, non_blocking=True)
-        V.step(stage)
-        for dst, src in zip(res_host, (V.path, V.len, V.bonus)):
-            dst.copy_(src, non_blocking=True)
+    def upload(s):
+        k = s % 2
+        copy_s.wait_event(free[k])                  # the step that last read this stage is done
+        with torch.cuda.stream(copy_s):
+            for dst, src in zip(stages[k].tensors(), pinned[s % N_DISTINCT]):
+                dst.copy_(src, non_blocking=True)
+        ready[k].record(copy_s)
 
-    for s in range(args.warmup):
-        e2e_step(s)
+    def e2e_run(first, count):
+        copy_s.wait_stream(comp)
+        upload(first)
+        for i in range(count):
+            s = first + i
+            if i + 1 < count:
+                upload(s + 1)
+            comp.wait_event(ready[s % 2])
+            V.step(stages[s % 2])
+            free[s % 2].record(comp)
+            for dst, src in zip(res_host, (V.path, V.len, V.bonus)):
+                dst.copy_(src, non_blocking=True)
+
+    e2e_run(0, args.warmup)
     torch.cuda.synchronize()
     HN.barrier(local)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for s in range(args.steps):
-        e2e_step(args.warmup + s)
+    e2e_run(args.warmup, args.steps)
     e1.record()
     torch.cuda.synchronize()
     HN.barrier(local)
+    assert np.array_equal(V.lens.cpu().numpy(), lens_np), "end-to-end arm: cache lengths diverged"
     e2e_el = HN.max_over_ranks(e0.elapsed_time(e1) * 1e-3, torch.device("cuda", local))
     e2e_rate = HN.whole_job_rate(args.steps, world, e2e_el)
 
