@@ -308,6 +308,18 @@ def test_accept_budget0_and_planted_paths():
             assert bonus[b] == st.argmax[b][st.planted[b][-1]]
 
 
+def test_accept_duplicate_sibling_tokens_take_the_lowest_index():
+    """Worked by hand.  Nodes 1 and 2 are both children of the root and both carry
+    token 5, the root's prediction; node 3 (token 7) hangs under node 1 and node 4
+    (token 9) under node 2, and the target predicts 7 after node 1 and 9 after node 2.
+    The lowest-index reading steps to node 1, then node 3: path [0, 1, 3], bonus 4
+    (the prediction after node 3).  Stepping to node 2 would give [0, 2, 4]."""
+    parents = [-1, 0, 0, 1, 2]
+    tokens = [8, 5, 5, 7, 9]
+    argmax = [5, 7, 9, 4, 6]
+    assert oracle.tree_accept(tokens, parents, argmax) == ([0, 1, 3], 3, 4)
+
+
 # ---------------------------------------------------------------- compaction
 def test_compaction_overlap_order():
     """path [0,2,3]: slot L+1 takes old L+2 and slot L+2 takes old L+3.  Copying
