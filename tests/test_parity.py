@@ -135,6 +135,22 @@ def test_accept_small_alphabet_many_matches(kd):
     assert rl.max() > 3
 
 
+def test_accept_duplicate_sibling_tokens(kd):
+    """Siblings may carry the same token (a 2-token alphabet, no resampling): the walk
+    takes the lowest-index matching child, as the oracle does."""
+    rng = np.random.default_rng(13)
+    B, n = 200, 70
+    parents = np.stack([W.draw_parents(rng, n, "branch", 4) for _ in range(B)])
+    tokens = rng.integers(0, 2, size=(B, n)).astype(np.int32)
+    argmax = rng.integers(0, 2, size=(B, n)).astype(np.int32)
+    path, ln, bonus = kd.kd_tree_accept(dev_i32(tokens), dev_i32(parents), dev_i32(argmax))
+    torch.cuda.synchronize()
+    rp, rl, rb = tree_accept_batch(tokens, parents, argmax)
+    assert np.array_equal(path.cpu().numpy(), rp) and np.array_equal(ln.cpu().numpy(), rl)
+    assert np.array_equal(bonus.cpu().numpy(), rb)
+    assert rl.max() > 4
+
+
 def test_accept_budget0_and_max_nodes(kd):
     rng = np.random.default_rng(12)
     for n in [1, 128]:
