@@ -3,12 +3,13 @@
  * DDTree speculative decoding for Multi-head Latent Attention (MLA) models.
  *
  * One verify step (sources are the pages' titles and sections):
+ *   0. kd_tree_build         the draft tree itself, best first from the drafter's
+ *                            per-depth candidates ("The Architecture of Pragmatic
+ *                            Ambition", "The Knowledge Architecture");
  *   1. kd_kv_write_nodes     the budget+1 node latents go to the next free slots,
  *                            root first ("The Architectural Keystone: Writing the
  *                            Model Header ...", "The Reasoning That Preceded the
  *                            Header");
- *   0. kd_tree_build         the draft tree itself, best first from the drafter's
- *                            per-depth candidates ("The Knowledge Architecture");
  *   2. kd_tree_build_mask    per-node ancestor bitmasks from the parent array
  *                            ("The Architecture of Pragmatic Ambition", "The
  *                            Knowledge Architecture": attention over the tree with
@@ -298,9 +299,12 @@ int kd_kv_write_nodes(kd_bf16_t* c_kv, kd_bf16_t* k_rope, int64_t kv_row_stride_
 /*
  * kd_tree_verify_attn_paged -- kd_tree_verify_attn over a paged cache.  page_size is
  * 64, 128 or 256 and pages_per_req at most 2047; the workspace is sized by
- * kd_verify_workspace_bytes(B, n, H, pages_per_req * page_size, kv_splits).  Page
- * ids outside [0, num_pages) read as zero rows (no fault); KD_EINVAL otherwise as
- * the contiguous call.
+ * kd_verify_workspace_bytes(B, n, H, pages_per_req * page_size, kv_splits);
+ * KD_EINVAL otherwise as the contiguous call.  This call does not check page ids:
+ * the caller keeps every id a request reads in [0, num_pages) (kd_kv_write_nodes_paged
+ * flags bad ids in the pages it writes).  A bad id never faults: an id below 0 or
+ * from num_pages up to 2^31 / page_size reads zero rows, and a larger one wraps in
+ * 32-bit row arithmetic and reads other rows of the pool.
  */
 int kd_tree_verify_attn_paged(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* q_rope,
                               const kd_bf16_t* c_pages, const kd_bf16_t* r_pages,
