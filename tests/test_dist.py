@@ -74,3 +74,23 @@ def test_algorithmic_work_formulas():
     assert c({"reasons": ["hw_slowdown"], "sm_mhz": 1900, "sm_max_mhz": 1965})
     assert not c({"reasons": ["sw_power_cap"], "sm_mhz": 1400, "sm_max_mhz": 1965})
     assert c({"reasons": [], "sm_mhz": 700, "sm_max_mhz": 1965})
+
+
+def test_flops_equal_visible_pairs_counted_from_the_masks():
+    """The roofline's FLOP count is 2 * H * (576 + 512) per visible (node, key) pair:
+    every node sees the L committed keys plus the set bits of its ancestor mask."""
+    import bench
+    import oracle
+    rng = np.random.default_rng(5)
+    for name in ["tiny", "kimi_single", "batched", "long", "loop"]:
+        cfg = W.CONFIGS[name]
+        st = W.draw_step(W.scaled(cfg, B=min(cfg.B, 6), H=1), 0, with_nodes=False)
+        lens = rng.integers(0, 5000, size=len(st.parents))
+        pairs = 0
+        for b, p in enumerate(st.parents):
+            bits = sum(bin(int(w)).count("1") for w in oracle.visibility_words(p).ravel())
+            pairs += len(p) * int(lens[b]) + bits
+        depths = [oracle.depths(p) for p in st.parents]
+        assert HN.attn_flops(lens, depths, 64) == 2.0 * 64 * (576 + 512) * pairs
+        for p, d in zip(st.parents, depths):                 # the bench's own depth walk
+            assert list(bench._depths(list(p))) == list(d)
