@@ -253,6 +253,36 @@ def _build(bug):
     return lambda: _replace(tb.tree_build, fn)
 
 
+# ---------------------------------------------------------------- whole step
+def _step(bug):
+    orig = oracle.step.verify_step
+
+    def fn(c_kv, k_rope, cache_lens, parents, tokens, argmax, q_abs, q_rope, scale,
+           node_ckv=None, node_krope=None, attn_nodes=None, with_attention=True):
+        c_in, r_in = c_kv, k_rope
+        if node_ckv is not None:
+            if bug == "write_next_slot":
+                c_kv, k_rope = c_kv.copy(), k_rope.copy()
+                for b in range(node_ckv.shape[0]):
+                    L = int(cache_lens[b])
+                    for k in range(node_ckv.shape[1]):
+                        c_kv[b, L + k + 1] = node_ckv[b, k]      # MUTANT
+                        k_rope[b, L + k + 1] = node_krope[b, k]
+            else:
+                c_kv, k_rope = cache.kv_write_nodes(c_kv, k_rope, cache_lens, node_ckv, node_krope)
+        vis = np.stack([tree.visibility_words(p) for p in parents])
+        out = lse = None
+        if with_attention:
+            src_c, src_r = (c_in, r_in) if bug == "attend_pre_write" else (c_kv, k_rope)  # MUTANT (one arm)
+            out, lse = att.tree_verify_attention(q_abs, q_rope, src_c, src_r, cache_lens, vis,
+                                                 scale, nodes=attn_nodes)
+        path, ln, bonus = acc.tree_accept_batch(tokens, parents, argmax)
+        c2, r2, lens2 = cache.kv_compact(c_kv, k_rope, cache_lens, path, ln)
+        return dict(out=out, lse=lse, vis=vis, path=path, len=ln, bonus=bonus,
+                    c_kv=c2, k_rope=r2, cache_lens=lens2, c_kv_pre=c_kv, k_rope_pre=k_rope)
+    return lambda: _replace(orig, fn)
+
+
 MUTANTS = {
     "attn_no_rope": _attention("no_rope"),
     "attn_scale_abs_only": _attention("scale_abs_only"),
@@ -286,6 +316,8 @@ MUTANTS = {
     "build_no_sibling": _build("no_sibling"),
     "build_sibling_own_score": _build("sibling_own_score"),
     "build_child_same_row": _build("child_same_row"),
+    "step_attend_pre_write": _step("attend_pre_write"),
+    "step_write_next_slot": _step("write_next_slot"),
 }
 
 

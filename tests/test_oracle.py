@@ -391,6 +391,50 @@ def test_verify_step_tiny_consistent_with_planted():
     assert np.isfinite(res["out"]).all() and np.isfinite(res["lse"]).all()
 
 
+def test_verify_step_attends_over_the_written_node_latents():
+    """Whole step with node latents, against a closed form built without the oracle's
+    cache functions.  With q = 0 every visible key scores 0, so out[b][i][h] is the mean
+    of the rows request b's node i sees -- committed slots [0, L) of the input cache and
+    the NODE LATENTS of its ancestors-or-self (written at slots L + k before attention:
+    "The Architectural Keystone ...", "The Reasoning That Preceded the Header") -- and
+    lse = ln |V|.  Slots at and past L hold garbage that must not be seen."""
+    rng = np.random.default_rng(21)
+    B, n, H = 2, 6, 2
+    lens = np.array([7, 3], np.int32)
+    parents = np.array([[-1, 0, 1, 0, 3, 4], [-1, 0, 0, 2, 2, 1]], np.int32)
+    cap = int(lens.max()) + n + 4
+    c_kv = rand_bf16((B, cap, 512), rng, std=1.0)            # garbage past L as well
+    k_rope = rand_bf16((B, cap, 64), rng, std=1.0)
+    node_c = rand_bf16((B, n, 512), rng, std=1.0)
+    node_r = rand_bf16((B, n, 64), rng, std=1.0)
+    zq_a = np.zeros((B, n, H, 512), np.uint16)
+    zq_r = np.zeros((B, n, H, 64), np.uint16)
+    tokens = np.arange(B * n, dtype=np.int32).reshape(B, n)
+    argmax = np.full((B, n), -1, np.int32)
+    argmax[0, 0], argmax[0, 3] = tokens[0, 3], tokens[0, 4]  # request 0 accepts 0 -> 3 -> 4
+    res = oracle.verify_step(c_kv, k_rope, lens, parents, tokens, argmax, zq_a, zq_r,
+                             1.0 / math.sqrt(192), node_ckv=node_c, node_krope=node_r)
+    C, NC = dec(c_kv).numpy(), dec(node_c).numpy()
+    for b in range(B):
+        L = int(lens[b])
+        for i in range(n):
+            anc, k = [], i
+            while k >= 0:                                     # ancestors-or-self by walking up
+                anc.append(k)
+                k = int(parents[b, k])
+            rows = np.concatenate([C[b, :L], NC[b, sorted(anc)]])
+            for h in range(H):
+                np.testing.assert_allclose(res["out"][b, i, h], rows.mean(0), rtol=1e-12, atol=1e-15)
+                assert abs(res["lse"][b, i, h] - math.log(L + len(anc))) < 1e-12
+        # node k sits at slot L + k after the write; the accepted path is gathered after it
+        assert np.array_equal(res["c_kv_pre"][b, L:L + n], node_c[b])
+        assert np.array_equal(res["k_rope_pre"][b, L:L + n], node_r[b])
+        m = int(res["len"][b])
+        assert np.array_equal(res["c_kv"][b, L:L + m], node_c[b, res["path"][b, :m]])
+        assert res["cache_lens"][b] == L + m
+    assert list(res["path"][0, :res["len"][0]]) == [0, 3, 4] and res["len"][1] == 1
+
+
 # ---------------------------------------------------------------- regression record
 def test_golden_tiny_regression():
     import json
