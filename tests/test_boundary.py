@@ -48,8 +48,10 @@ def test_workspace_bytes(lib):
     from tree_speculative_decoding_kd_b200 import kd
     # no split: control block only
     assert kd.kd_verify_workspace_bytes(1, 8, 16, 300, 1) == 256
-    rows = 8 * 65 * 64
-    want = 256 + ((rows * 3 * 4 + 255) // 256) * 256 + rows * 3 * 512 * 4
+    # control block, tickets [B * mtiles][2] int32, partial lse [S][rows], partials [S][rows][512]
+    rows, mtiles = 8 * 65 * 64, -(-65 * 64 // 128)
+    up = lambda x: -(-x // 256) * 256  # noqa: E731
+    want = 256 + up(8 * mtiles * 8) + up(rows * 3 * 4) + rows * 3 * 512 * 4
     assert kd.kd_verify_workspace_bytes(8, 65, 64, 32833, 3) == want
     assert kd.kd_verify_workspace_bytes(8, 65, 64, 32833, 0) >= 256
     for bad in [(0, 8, 16, 300, 0), (1, 0, 16, 300, 0), (1, 129, 16, 300, 0), (1, 8, 0, 300, 0),

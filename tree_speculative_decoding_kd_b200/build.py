@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libkdverify.so")
 
-SOURCES = ["kd_tree.cu", "kd_attn_simt.cu", "kd_attn_combine.cu", "kd_attn_tc.cu", "kd_argmax.cu", "kd_tree_build.cu"]
+SOURCES = ["kd_tree.cu", "kd_attn_simt.cu", "kd_attn_tc.cu", "kd_argmax.cu", "kd_tree_build.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I" + INCLUDE, "-I" + CSRC]
