@@ -34,15 +34,17 @@
 //       neither loaded nor multiplied.  Two 4-warp groups apply the rare O rescale
 //       and write the normalised output straight from registers to global memory.
 //
-// The kernel is persistent: one cluster per SM pair, each walking its share of
-// the units (requests ranked longest first, waves of units dealt to the clusters
-// in alternating order).  Units overlap at their boundaries: the next unit's Q
-// streams in behind the current unit's last K stages, and the output of one unit
-// is written while the next one's scores are computed.  Key partitions of one M
-// tile (split-KV, for short batches) are merged inside the same launch: each
-// partition stores a normalised fp32 partial, bumps a per-tile ticket, and after
-// its last unit every cluster merges its share of the rows of each tile it worked
-// on once that tile's ticket is complete (log-sum-exp identity).
+// The kernel is persistent: one cluster per SM pair.  Units are handed out
+// dynamically from a global counter in longest-request-first order; each cluster's
+// QK producer claims the next one while its current unit's last tile loads and
+// publishes it to every role of both CTAs through a small ring in shared memory.
+// Units overlap at their boundaries: the next unit's Q streams in behind the
+// current unit's last K stages, and the output of one unit is written while the
+// next one's scores are computed.  Key partitions of one M tile (split-KV, for
+// short batches) are merged inside the same launch: each partition stores a
+// normalised fp32 partial and bumps a per-tile ticket; after its last unit every
+// CTA merges a fixed share of the rows once their tile's ticket is complete
+// (log-sum-exp identity).
 //
 // attn_tc_kernel<true> reads a paged cache instead: each 256-key K stage arrives as
 // one TMA box per page and each 64-key V group as one box inside a page, from the
@@ -117,12 +119,17 @@ enum Bar {
   EVENT = O_FREE + 1,                   // PV: rescale or end-of-unit event for the epilogue
   CORR_DONE = EVENT + 1,                // PV: rescale applied (256 arrivals)
   PV_DRAIN = CORR_DONE + 1,             // PV: all issued PV MMAs done (before a rescale)
-  NBAR = PV_DRAIN + 1
+  SCHED_FULL = PV_DRAIN + 1,            // both: schedule slot k % NS published
+  SCHED_EMPTY = SCHED_FULL + 4,         // QK: schedule slot read by all five consumers
+  NBAR = SCHED_EMPTY + 4
 };
+constexpr int NS = 4;                   // schedule ring depth
+constexpr int SCHED_READERS = 5;        // QK MMA, QK softmax, PV producer, PV MMA, PV epilogue
 constexpr int OFF_TMEM = 512;           // u32 TMEM base
 constexpr int OFF_ABORT = 516;          // u32 abort flag
 constexpr int OFF_EVTYPE = 520;         // u32 event type (1 rescale, 2 end of unit)   [PV]
 constexpr int OFF_EVTILE = 524;         // u32 P slot of a rescale event               [PV]
+constexpr int OFF_SCHED = 544;          // i64 [NS] unit ranks of this cluster (-1: no more work)
 constexpr int OFF_ORDER = 1024;         // i32 [LPT_MAX] requests by length
 constexpr int OFF_MFIN = 2048;          // f32 [128] final running max (log2)          [PV, remote]
 constexpr int OFF_LFIN = 2560;          // f32 [128] final running sum                 [PV, remote]
@@ -137,7 +144,8 @@ constexpr int K_OFF = STG_OFF + 2 * PSLOT;
 constexpr int QK_END = K_OFF + NK * KCHUNK;
 constexpr int P_OFF = CTRL;
 constexpr int V_OFF = P_OFF + 2 * PSLOT;
-constexpr int PV_END = V_OFF + NVG * VG;
+constexpr int EPI_OFF = V_OFF + NVG * VG;                 // epilogue staging, 2 KB per worker warp
+constexpr int PV_END = EPI_OFF + 8 * 2048;
 constexpr int PT_OFF = QK_END > PV_END ? QK_END : PV_END;   // paged caches: the unit's page slice
 constexpr int PT_MAX = 2048;                                  // int32 entries (8 KB)
 constexpr int SMEM_BYTES = PT_OFF + PT_MAX * 4 + 1024;
@@ -159,6 +167,7 @@ struct Params {
   float* part_lse;                // [splits][B * n * H]
   int32_t* tickets;               // [B * mtiles][2]: partitions stored, merges done
   int32_t* err;
+  unsigned long long* sched;      // [0] next unit rank to hand out, [1] clusters done (self-resetting)
   int64_t cap;                    // logical slots per request (pages_per_req * P when paged)
   int64_t units;                  // B * mtiles * splits
   int B, n, H, W, mtiles, splits, clusters;
@@ -240,13 +249,6 @@ struct Unit {
   bool valid;
 };
 
-// Rank of the k-th unit of cluster c: waves of `clusters` units are dealt in
-// alternating directions, so the long units at the front of each wave and the
-// short ones at its back even out across clusters.
-__device__ __forceinline__ int64_t unit_rank(const Params& p, int c, int k) {
-  return (int64_t)k * p.clusters + ((k & 1) ? (p.clusters - 1 - c) : c);
-}
-
 // Unit of rank r: requests in `order` (longest first), then key partition, then M
 // tile (the M tiles of one partition read the same keys and run side by side).
 __device__ __forceinline__ Unit unit_at(const Params& p, const int* order, int64_t r) {
@@ -267,13 +269,36 @@ __device__ __forceinline__ Unit unit_at(const Params& p, const int* order, int64
   return u;
 }
 
-// First rank >= k of cluster c whose unit has key tiles (-1 if none).
-__device__ __forceinline__ int next_busy_unit(const Params& p, const int* order, int c, int k) {
-  for (;; ++k) {
-    const int64_t r = unit_rank(p, c, k);
-    if (r >= p.units) return -1;
-    if (unit_at(p, order, r).ntiles > 0) return k;
+// ---------------------------------------------------------------- schedule ring
+// Units are handed out dynamically: the QK producer claims ranks from a global
+// counter (longest requests first, see unit_at), skips those with no key tiles and
+// publishes the k-th rank of its cluster in slot k % NS of a ring that both CTAs
+// hold (the peer's copy written remotely); -1 ends the cluster's work.  Every role
+// reads the ring in order and frees each slot once it has read it.
+__device__ __forceinline__ volatile int64_t* sched_slots(uint8_t* gbase) {
+  return reinterpret_cast<volatile int64_t*>(gbase + OFF_SCHED);
+}
+
+// Frees slot s from a role of this CTA (QK) or of the peer (PV).
+__device__ __forceinline__ void sched_release(const Ctx& cx, int s, bool remote) {
+  if (remote) mbar_arrive_remote(map_to_rank(cx.bar(SCHED_EMPTY + s), cx.peer));
+  else mbar_arrive(cx.bar(SCHED_EMPTY + s));
+}
+
+// Rank the whole warp learns from lane 0's claims: the next rank with key tiles
+// (requests whose cache does not fit raise KD_DEV_CACHE_FULL once), or -1.
+__device__ __forceinline__ int64_t claim_unit(const Params& p, const int* order, int64_t first) {
+  int64_t r = first;
+  if ((threadIdx.x & 31) == 0) {
+    while (r < p.units) {
+      const Unit u = unit_at(p, order, r);
+      if (u.ntiles > 0) break;
+      if (!u.valid && u.mt == 0 && u.sp == 0) raise_dev_error(p.err, KD_DEV_CACHE_FULL);
+      r = (int64_t)atomicAdd(p.sched, 1ull);
+    }
+    if (r >= p.units) r = -1;
   }
+  return __shfl_sync(0xffffffffu, r, 0);
 }
 
 // Cache row of request-relative key `key` of a paged cache (the unit's page-table
@@ -312,22 +337,35 @@ __device__ __forceinline__ bool request_pages_ok(const Params& p, int b, int64_t
 }
 
 // ====================================================================== QK CTA roles
-// TMA producer (whole warp; lane 0 issues): per unit, the Q latent through four
-// ring stages, the rope chunk of Q, then the K stages of every tile.
+// TMA producer and scheduler (whole warp; lane 0 issues): claims the cluster's
+// units and publishes them, then per unit loads the Q latent through four ring
+// stages, the rope chunk of Q, and the K stages of every tile.
 template <bool PAGED>
-__device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, const int* order, int cid,
+__device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, const int* order, uint8_t* gbase,
                                             int32_t* ptab, const CUtensorMap* tm_qa,
                                             const CUtensorMap* tm_qr, const CUtensorMap* tm_c,
                                             const CUtensorMap* tm_r) {
   const int lane = threadIdx.x & 31;
   const uint32_t base = cx.base;
+  volatile int64_t* slots = sched_slots(gbase);
+  const uint32_t peer_slots = map_to_rank(base + OFF_SCHED, cx.peer);
   uint32_t it = 0, uq = 0;
   bool ok = true;
-  for (int k = 0; ok; ++k) {
-    const int64_t r = unit_rank(p, cid, k);
-    if (r >= p.units) break;
+  int64_t r = claim_unit(p, order, lane == 0 ? (int64_t)atomicAdd(p.sched, 1ull) : 0);
+  for (int k = 0;; ++k) {
+    // publish the k-th unit (or the end) once every role has read slot k - NS
+    const int sl = k % NS;
+    if (!(ok = wait_warp(cx, cx.bar(SCHED_EMPTY + sl), ((k / NS) & 1) ^ 1))) break;
+    if (lane == 0) {
+      slots[sl] = r;
+      st_cluster_u32(peer_slots + sl * 8, (uint32_t)(uint64_t)r);
+      st_cluster_u32(peer_slots + sl * 8 + 4, (uint32_t)((uint64_t)r >> 32));
+      mbar_arrive(cx.bar(SCHED_FULL + sl));
+      mbar_arrive_remote(map_to_rank(cx.bar(SCHED_FULL + sl), cx.peer));
+    }
+    __syncwarp();
+    if (r < 0) break;
     const Unit u = unit_at(p, order, r);
-    if (u.ntiles == 0) continue;
     const int qrow0 = u.b * p.n * p.H + u.mt * BM;
     for (int q = 0; q < QSTAGES; ++q, ++it) {
       const uint32_t st = it % NK;
@@ -353,6 +391,7 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, cons
       stage_pages(p, ptab, u.b, page0, pend < p.pages_per_req ? pend : p.pages_per_req);
     }
     const int64_t krow0 = (int64_t)u.b * p.cap + u.kbeg;
+    int64_t claimed = 0;
     for (int t = 0; t < u.ntiles && ok; ++t) {
       const int32_t krow = (int32_t)(krow0 + (int64_t)t * BQ);
       int32_t prow[4];                // paged: the cache rows of the tile's (at most 4) pages
@@ -362,6 +401,8 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, cons
           prow[i] = (i << p.page_shift) < BQ
                         ? paged_row(ptab, page0, p, u.kbeg + (int64_t)t * BQ + (i << p.page_shift)) : 0;
       }
+      // claim the next unit during the last tile, so the claim's latency is hidden
+      if (t == u.ntiles - 1 && lane == 0) claimed = (int64_t)atomicAdd(p.sched, 1ull);
       for (int c = 0; c < NCHUNK; ++c, ++it) {
         const uint32_t st = it % NK;
         if (!(ok = wait_warp(cx, cx.bar(K_EMPTY + st), ((it / NK) & 1u) ^ 1u))) break;
@@ -381,28 +422,37 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, cons
         }
       }
     }
+    if (!ok) break;
+    r = claim_unit(p, order, claimed);
   }
   // every armed copy must land before the CTA may leave (bounded, even after an abort)
   if (lane == 0) {
     for (uint32_t j = (it > NK ? it - NK : 0); j < it; ++j)
       wait_bar(cx, cx.bar(K_FULL + j % NK), (j / NK) & 1u, false, true);
     if (uq > 0) wait_bar(cx, cx.bar(ROPE_FULL), (uq - 1) & 1u, false, true);
+    // the last cluster to run out of work returns the counter to zero for the next launch
+    if (atomicAdd(p.sched + 1, 1ull) == (unsigned long long)(p.clusters - 1)) {
+      p.sched[0] = 0ull;
+      p.sched[1] = 0ull;
+    }
   }
   __syncwarp();
 }
 
 // MMA issuer: S = Q K^T per tile (A from TMEM for chunks 0..7, from shared memory
 // for the rope chunk).
-__device__ __forceinline__ void qk_mma(const Ctx& cx, const Params& p, const int* order, int cid,
+__device__ __forceinline__ void qk_mma(const Ctx& cx, const Params& p, const int* order, uint8_t* gbase,
                                        uint32_t tmem) {
   const uint32_t base = cx.base;
+  volatile int64_t* slots = sched_slots(gbase);
   uint32_t it = 0, ts = 0, uq = 0;
   bool ok = true;
   for (int k = 0; ok; ++k) {
-    const int64_t r = unit_rank(p, cid, k);
-    if (r >= p.units) break;
+    if (!(ok = wait_bar(cx, cx.bar(SCHED_FULL + k % NS), (k / NS) & 1, true))) break;
+    const int64_t r = slots[k % NS];
+    sched_release(cx, k % NS, false);
+    if (r < 0) break;
     const Unit u = unit_at(p, order, r);
-    if (u.ntiles == 0) continue;
     it += QSTAGES;                              // Q stages are consumed by the softmax groups
     if (!(ok = wait_bar(cx, cx.bar(QT_FULL), uq & 1u) && wait_bar(cx, cx.bar(ROPE_FULL), uq & 1u))) break;
     tc_fence_after();
@@ -511,8 +561,8 @@ __device__ __forceinline__ bool emit_p(const Ctx& cx, uint8_t* gbase, const floa
 
 // Softmax groups: thread (g, r) owns row r and key columns [64 g, 64 g + 64) of
 // every 128-key half of every tile.
-__device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const int* order, int cid,
-                                           uint8_t* gbase, uint32_t tmem) {
+__device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const int* order, uint8_t* gbase,
+                                           uint32_t tmem) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = (warp - 2) >> 2;
   const int quad = warp & 3;
@@ -521,37 +571,42 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
   const int n = p.n, H = p.H, rows_req = n * H, W = p.W;
   // two exchange buffers, alternating by tile, so a tile's writes never meet the
   // previous tile's reads
-  float* const xchb[2] = {reinterpret_cast<float*>(gbase + OFF_XCH0), reinterpret_cast<float*>(gbase + OFF_XCH)};
+  const uint32_t xch0 = cx.base + OFF_XCH0;               // buffer b at xch0 + b * 1024
   const uint32_t peer_p = map_to_rank(cx.base + P_OFF, cx.peer);
   const uint32_t peer_ctrl = map_to_rank(cx.base, cx.peer);
 
+  volatile int64_t* slots = sched_slots(gbase);
   uint32_t pos = 0, ts = 0, pc = 0, nq = 0, ns = 0;
-  bool ok = true;
-  int kq = next_busy_unit(p, order, cid, 0);            // the unit whose Q is copied next
-  if (kq >= 0) ok = copy_q(cx, gbase, lane_addr, 0, g, r);
+  bool ok = wait_group(cx, cx.bar(SCHED_FULL), 0, true);
+  if (ok && slots[0] >= 0) ok = copy_q(cx, gbase, lane_addr, 0, g, r);     // the first unit's Q
   for (int k = 0; ok; ++k) {
-    const int64_t rk = unit_rank(p, cid, k);
-    if (rk >= p.units) break;
+    if (!(ok = wait_group(cx, cx.bar(SCHED_FULL + k % NS), (k / NS) & 1, true))) break;
+    const int64_t rk = slots[k % NS];
+    named_bar_sync(1, GROUP);                   // every thread has read the slot
+    if (threadIdx.x == 64) sched_release(cx, k % NS, false);
+    if (rk < 0) break;
     const Unit u = unit_at(p, order, rk);
-    if (!u.valid) {
-      if (threadIdx.x == 64 && u.mt == 0 && u.sp == 0) raise_dev_error(p.err, KD_DEV_CACHE_FULL);
-      continue;
-    }
     float m_ref = -INFINITY, l_part = 0.f;
-    if (u.ntiles > 0) {
-      const int R = u.mt * BM + r;
-      const bool valid_row = R < rows_req;
-      const int node = valid_row ? R / H : 0;
-      uint32_t w[4];
+    {
+      // this row's node (its mask is read again where a tile reaches the tree slots)
+      const uint32_t* vrow;
+      {
+        const int R = u.mt * BM + r;
+        const bool valid_row = R < rows_req;
+        const int node = valid_row ? R / H : 0;
+        vrow = p.vis + ((size_t)u.b * n + node) * W;
+        if (g == 0 && valid_row && u.sp == 0 && (R % H) == 0) {
+          uint32_t w[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) w[q] = q < W ? p.vis[((size_t)u.b * n + node) * W + q] : 0u;
-      if (g == 0 && valid_row && u.sp == 0 && (R % H) == 0) {
-        const int depth = __popc(w[0]) + __popc(w[1]) + __popc(w[2]) + __popc(w[3]) - 1;
-        if (!(w[0] & 1u) || !((mask_word(w, node >> 5) >> (node & 31)) & 1u))
-          raise_dev_error(p.err, KD_DEV_BAD_MASK);
-        if (p.positions && p.positions[(size_t)u.b * n + node] != (int32_t)(u.L + depth))
-          raise_dev_error(p.err, KD_DEV_BAD_POSITION);
+          for (int q = 0; q < 4; ++q) w[q] = q < W ? vrow[q] : 0u;
+          const int depth = __popc(w[0]) + __popc(w[1]) + __popc(w[2]) + __popc(w[3]) - 1;
+          if (!(w[0] & 1u) || !((mask_word(w, node >> 5) >> (node & 31)) & 1u))
+            raise_dev_error(p.err, KD_DEV_BAD_MASK);
+          if (p.positions && p.positions[(size_t)u.b * n + node] != (int32_t)(u.L + depth))
+            raise_dev_error(p.err, KD_DEV_BAD_POSITION);
+        }
       }
+      const int rel0 = (int)(u.kbeg - u.L);     // first key of the unit relative to slot L
       for (int t = 0; t < u.ntiles && ok; ++t, ++ts) {
         if (!(ok = wait_group(cx, cx.bar(S_FULL), ts & 1u))) break;
         tc_fence_after();
@@ -574,8 +629,11 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           // key index relative to the first tree slot L (fits 32 bits: keys < 2^31)
-          const int kt = (int)(u.kbeg - u.L) + t * BQ + h * BN + g * 64;
+          const int kt = rel0 + t * BQ + h * BN + g * 64;
           if (kt + 64 > 0) {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) w[q] = q < W ? vrow[q] : 0u;
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
               const int kk = kt + c;
@@ -596,10 +654,10 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
             mx[2] = fmax3(mx[2], x[h][c + 2], x[h][c + 6]);
             mx[3] = fmax3(mx[3], x[h][c + 3], x[h][c + 7]);
           }
-        float* xch = xchb[ts & 1];
-        xch[g * BM + r] = max4(mx[0], mx[1], mx[2], mx[3]);
+        const uint32_t xch = xch0 + (ts & 1) * 1024;
+        st_shared_f32(xch + (g * BM + r) * 4, max4(mx[0], mx[1], mx[2], mx[3]));
         named_bar_sync(1, GROUP);
-        const float tmax = fmaxf(xch[r], xch[BM + r]) * p.scale_log2;
+        const float tmax = fmaxf(ld_shared_f32(xch + r * 4), ld_shared_f32(xch + (BM + r) * 4)) * p.scale_log2;
         float alpha = 1.f;
         bool rescale_row = false;
         if (tmax > m_ref + RESCALE_THRESHOLD) {
@@ -617,9 +675,11 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
                     l_part);
         if (ok && t == u.ntiles - 1) {
           // the last S of this unit is out of TMEM, so once its MMAs are done the next
-          // unit's Q may replace this one's (done with half the scores already spent)
-          const int knext = next_busy_unit(p, order, cid, k + 1);
-          if (knext >= 0)
+          // unit's Q (if the schedule has one) may replace this one's; done with half
+          // the scores already spent
+          const int kn = k + 1;
+          ok = wait_group(cx, cx.bar(SCHED_FULL + kn % NS), (kn / NS) & 1, true);
+          if (ok && slots[kn % NS] >= 0)
             ok = wait_group(cx, cx.bar(Q_FREE), nq & 1u) &&
                  copy_q(cx, gbase, lane_addr, pos + QSTAGES + NCHUNK * (uint32_t)u.ntiles, g, r);
         }
@@ -633,10 +693,10 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
     }
     // final row statistics for the epilogue: l = both groups' partial sums (in the
     // exchange buffer the next tile will use)
-    float* xch = xchb[ts & 1];
-    xch[g * BM + r] = l_part;
+    const uint32_t xch = xch0 + (ts & 1) * 1024;
+    st_shared_f32(xch + (g * BM + r) * 4, l_part);
     named_bar_sync(1, GROUP);
-    const float l_row = xch[r] + xch[BM + r];
+    const float l_row = ld_shared_f32(xch + r * 4) + ld_shared_f32(xch + (BM + r) * 4);
     if (ns > 0 && !(ok = wait_group(cx, cx.bar(STATS_FREE), (ns - 1) & 1u))) break;
     if (g == 0) {
       st_cluster_u32(peer_ctrl + OFF_MFIN + r * 4, __float_as_uint(m_ref));
@@ -665,16 +725,19 @@ __device__ __forceinline__ int group_keys(int64_t kbeg, int64_t nkeys, int t, in
 }
 
 template <bool PAGED>
-__device__ __forceinline__ void pv_producer(const Ctx& cx, const Params& p, const int* order, int cid,
+__device__ __forceinline__ void pv_producer(const Ctx& cx, const Params& p, const int* order, uint8_t* gbase,
                                             int32_t* ptab, const CUtensorMap* tm_v) {
   const int lane = threadIdx.x & 31;
+  volatile int64_t* slots = sched_slots(gbase);
   bool ok = true;
   uint32_t gi = 0;
   for (int k = 0; ok; ++k) {
-    const int64_t r = unit_rank(p, cid, k);
-    if (r >= p.units) break;
+    if (!(ok = wait_warp(cx, cx.bar(SCHED_FULL + k % NS), (k / NS) & 1, true))) break;
+    const int64_t r = slots[k % NS];
+    __syncwarp();
+    if (lane == 0) sched_release(cx, k % NS, true);
+    if (r < 0) break;
     const Unit u = unit_at(p, order, r);
-    if (u.ntiles == 0) continue;
     const int page0 = PAGED ? (int)(u.kbeg >> p.page_shift) : 0;
     if (PAGED) {
       const int64_t kend = u.kbeg + (int64_t)u.ntiles * BQ;
@@ -706,17 +769,20 @@ __device__ __forceinline__ void pv_producer(const Ctx& cx, const Params& p, cons
   __syncwarp();
 }
 
-__device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int* order, int cid,
-                                       uint8_t* gbase, uint32_t tmem) {
+__device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int* order, uint8_t* gbase,
+                                       uint32_t tmem) {
   const int lane = threadIdx.x & 31;
   volatile uint32_t* ctrl = reinterpret_cast<volatile uint32_t*>(gbase);
+  volatile int64_t* slots = sched_slots(gbase);
   bool ok = true;
   uint32_t gi = 0, pc = 0, vu = 0, nres = 0, nd = 0;
   for (int k = 0; ok; ++k) {
-    const int64_t r = unit_rank(p, cid, k);
-    if (r >= p.units) break;
+    if (!(ok = wait_warp(cx, cx.bar(SCHED_FULL + k % NS), (k / NS) & 1, true))) break;
+    const int64_t r = slots[k % NS];
+    __syncwarp();
+    if (lane == 0) sched_release(cx, k % NS, true);
+    if (r < 0) break;
     const Unit u = unit_at(p, order, r);
-    if (!u.valid) continue;
     // the epilogue must have read the previous unit's O before it is overwritten
     if (vu > 0 && !(ok = wait_warp(cx, cx.bar(O_FREE), (vu - 1) & 1u))) break;
     for (int t = 0; t < 2 * u.ntiles && ok; ++t, ++pc) {      // P tiles of 128 keys
@@ -775,8 +841,7 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int
     }
     if (!ok) break;
     if (lane == 0) {
-      if (u.ntiles > 0) tc_commit(cx.bar(O_DONE));
-      else mbar_arrive(cx.bar(O_DONE));
+      tc_commit(cx.bar(O_DONE));
       ctrl[OFF_EVTYPE >> 2] = 2u;
       mbar_arrive(cx.bar(EVENT));
     }
@@ -790,9 +855,32 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int
   __syncwarp();
 }
 
+// Each lane holds 64 bytes (16 words) of its own row; the warp moves its 32 rows
+// through its 2 KB staging slot so that every global store instruction covers 8
+// rows x 64 contiguous bytes (row r of the warp goes to dst0 + r * pitch; rows from
+// nrows on are not written).  The slot's 16-byte pieces are swizzled by row so
+// that neither the row-wise writes nor the column-wise reads conflict on banks.
+__device__ __forceinline__ void warp_store_rows(uint32_t stg, const uint32_t (&w)[16], uint8_t* dst0,
+                                                int64_t pitch, int nrows) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();                                 // the previous round's reads are done
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    st_shared_v4(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2],
+                 w[4 * c + 3]);
+  __syncwarp();
+  const int ch = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int row = (lane >> 2) + 8 * j;
+    const uint4 v = ld_shared_v4(stg + row * 64 + ((ch ^ ((row >> 1) & 3)) << 4));
+    if (row < nrows) st_global_v4(dst0 + row * pitch + ch * 16, v.x, v.y, v.z, v.w);
+  }
+}
+
 // Correction / epilogue groups: thread (g, r) owns row r, O columns [256 g, 256 g + 256).
-__device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, const int* order, int cid,
-                                            uint8_t* gbase, uint32_t tmem, bool paged) {
+__device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, const int* order, uint8_t* gbase,
+                                            uint32_t tmem, bool paged) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = (warp - 2) >> 2;
   const int quad = warp & 3;
@@ -802,13 +890,16 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
   const volatile float* fctrl = reinterpret_cast<const volatile float*>(gbase);
   const uint32_t peer_ctrl = map_to_rank(cx.base, cx.peer);
   const int rows_req = p.n * p.H;
+  volatile int64_t* slots = sched_slots(gbase);
   bool ok = true;
   uint32_t nev = 0, vu = 0;
   for (int k = 0; ok; ++k) {
-    const int64_t rk = unit_rank(p, cid, k);
-    if (rk >= p.units) break;
+    if (!(ok = wait_group(cx, cx.bar(SCHED_FULL + k % NS), (k / NS) & 1, true))) break;
+    const int64_t rk = slots[k % NS];
+    named_bar_sync(1, GROUP);
+    if (threadIdx.x == 64) sched_release(cx, k % NS, true);
+    if (rk < 0) break;
     const Unit u = unit_at(p, order, rk);
-    if (!u.valid) continue;
     const bool pages_ok = !paged || request_pages_ok(p, u.b, u.nkeys);
     while (true) {
       if (!(ok = wait_group(cx, cx.bar(EVENT), nev & 1u))) break;
@@ -840,52 +931,42 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
     const int R = u.mt * BM + r;
     const bool write = pages_ok && R < rows_req;
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    const bool have_o = u.ntiles > 0;
     const int64_t grow = (int64_t)u.b * rows_req + R;
-    if (p.splits == 1) {
-      uint16_t* dst = p.out + grow * KD_D_C + g * 256;
-      for (int c = 0; c < 256 / 64; ++c) {
-        uint32_t v[64];
-        if (have_o) {
-          tmem_ld64(lane_addr + c * 64, v);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int q = 0; q < 64; ++q) v[q] = 0u;
-        }
-        if (write) {
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            st_global_v4(dst + c * 64 + q * 8,
-                         pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv),
-                         pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv),
-                         pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv),
-                         pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv));
-        }
+    // this warp's 32 rows: the first one, and how many of them exist
+    const int R0w = u.mt * BM + quad * 32;
+    const int nrows = pages_ok ? min(max(rows_req - R0w, 0), 32) : 0;
+    const int64_t grow0 = (int64_t)u.b * rows_req + R0w;
+    const uint32_t stg = cx.base + EPI_OFF + (warp - 2) * 2048;
+    uint8_t* dst0 = p.splits == 1
+                        ? reinterpret_cast<uint8_t*>(p.out + grow0 * KD_D_C + g * 256)
+                        : reinterpret_cast<uint8_t*>(p.part_o + ((int64_t)u.sp * p.B * rows_req + grow0) * KD_D_C + g * 256);
+    for (int c = 0; c < 256 / 64; ++c) {
+      uint32_t v[64];
+      tmem_ld64(lane_addr + c * 64, v);
+      tmem_wait_ld();
+      if (c == 256 / 64 - 1) {                  // every TMEM read of this unit is done
+        tc_fence_before();
+        mbar_arrive(cx.bar(O_FREE));
       }
-    } else {
-      float* dst = p.part_o + ((int64_t)u.sp * p.B * rows_req + grow) * KD_D_C + g * 256;
-      for (int c = 0; c < 256 / 64; ++c) {
-        uint32_t v[64];
-        if (have_o) {
-          tmem_ld64(lane_addr + c * 64, v);
-          tmem_wait_ld();
-        } else {
+      if (p.splits == 1) {                      // bf16: two rounds of 32 columns
 #pragma unroll
-          for (int q = 0; q < 64; ++q) v[q] = 0u;
-        }
-        if (write) {
+        for (int h = 0; h < 2; ++h) {
+          uint32_t w[16];
 #pragma unroll
           for (int q = 0; q < 16; ++q)
-            st_global_v4(dst + c * 64 + q * 4, __float_as_uint(__uint_as_float(v[4 * q]) * inv),
-                         __float_as_uint(__uint_as_float(v[4 * q + 1]) * inv),
-                         __float_as_uint(__uint_as_float(v[4 * q + 2]) * inv),
-                         __float_as_uint(__uint_as_float(v[4 * q + 3]) * inv));
+            w[q] = pack_bf16x2(__uint_as_float(v[32 * h + 2 * q]) * inv, __uint_as_float(v[32 * h + 2 * q + 1]) * inv);
+          warp_store_rows(stg, w, dst0 + (c * 64 + h * 32) * 2, KD_D_C * 2, nrows);
+        }
+      } else {                                  // fp32: four rounds of 16 columns
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          uint32_t w[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) w[q] = __float_as_uint(__uint_as_float(v[16 * h + q]) * inv);
+          warp_store_rows(stg, w, dst0 + (c * 64 + h * 16) * 4, KD_D_C * 4, nrows);
         }
       }
     }
-    tc_fence_before();
-    mbar_arrive(cx.bar(O_FREE));
     if (write && g == 0) {
       const float lse_v = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       if (p.splits == 1) p.lse[grow] = lse_v;
@@ -905,86 +986,105 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
 }
 
 // ====================================================================== split-KV merge
-// After its last unit, each CTA of a cluster merges its share of the rows of every
-// M tile whose partition it worked on: partition sp of a tile owns rows
-// [sp R / S, (sp+1) R / S) of the tile's R rows, split between the two CTAs, one
-// warp per row and 16 latent columns per lane:
+// Partition sp of request b covers QK tiles [sp T / S, (sp+1) T / S) of its T tiles;
+// partitions without tiles are never scheduled and store nothing.
+__device__ __forceinline__ bool partition_busy(int64_t T, int sp, int S) {
+  return (int64_t)(sp + 1) * T / S > (int64_t)sp * T / S;
+}
+
+// After its last unit, each CTA merges a fixed share of all rows (cluster c takes
+// rows [c R / G, (c+1) R / G) of the R = B n H rows, split between its two CTAs),
+// one M tile at a time once that tile's ticket shows every busy partition stored,
+// one warp per row and 16 latent columns per lane:
 //   LSE = ln sum_s exp(lse_s),   out = sum_s exp(lse_s - LSE) o_s.
-__device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, const int* order, int cid,
-                                             uint32_t rank, bool paged) {
+// The merged-row count on the tile's second ticket word tells the last merger to
+// return both words to zero for the next launch.
+__device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, int cid, uint32_t rank,
+                                             bool paged) {
   const int tid = threadIdx.x - 64;
   const int wid = tid >> 5, lane = threadIdx.x & 31;
   const int rows_req = p.n * p.H, S = p.splits;
   const int64_t rows_all = (int64_t)p.B * rows_req;
-  for (int k = 0;; ++k) {
-    const int64_t rk = unit_rank(p, cid, k);
-    if (rk >= p.units) break;
-    const Unit u = unit_at(p, order, rk);
-    if (!u.valid) continue;
-    int32_t* ticket = p.tickets + 2 * ((int64_t)u.b * p.mtiles + u.mt);
-    // wait until every partition of the tile has stored its partial
-    bool ok = true;
-    if (tid == 0) {
-      uint64_t t0 = 0;
-      for (uint32_t spin = 1; ld_acquire_gpu(ticket) < S; ++spin) {
-        if ((spin & 63u) == 0u) {
-          if (*cx.abort_flag) { ok = false; break; }
-          const uint64_t t = globaltimer();
-          if (t0 == 0) t0 = t;
-          else if (t - t0 > WAIT_LIMIT_NS) { abort_pair(cx); ok = false; break; }
+  const int64_t lo = (int64_t)cid * rows_all / p.clusters, hi = (int64_t)(cid + 1) * rows_all / p.clusters;
+  const int64_t mid = (lo + hi) / 2;
+  const int64_t a = rank == 0 ? lo : mid, e = rank == 0 ? mid : hi;
+  for (int64_t row0 = a; row0 < e;) {
+    const int b = (int)(row0 / rows_req);
+    const int R0 = (int)(row0 - (int64_t)b * rows_req);
+    const int mt = R0 / BM;
+    const int rows_in = rows_req - mt * BM < BM ? rows_req - mt * BM : BM;
+    const int64_t tile_end_g = (int64_t)b * rows_req + mt * BM + rows_in;
+    const int64_t row1 = tile_end_g < e ? tile_end_g : e;
+    const int64_t L = p.cache_lens[b];
+    const bool valid = L >= 0 && L + p.n <= p.cap;
+    if (valid) {
+      const int64_t nkeys = L + p.n;
+      const int64_t T = (nkeys + BQ - 1) / BQ;
+      int busy = 0;
+      for (int s = 0; s < S; ++s) busy += partition_busy(T, s, S);
+      int32_t* ticket = p.tickets + 2 * ((int64_t)b * p.mtiles + mt);
+      // wait until every busy partition of the tile has stored its partial
+      bool ok = true;
+      if (tid == 0) {
+        uint64_t t0 = 0;
+        for (uint32_t spin = 1; ld_acquire_gpu(ticket) < busy; ++spin) {
+          if ((spin & 63u) == 0u) {
+            if (*cx.abort_flag) { ok = false; break; }
+            const uint64_t t = globaltimer();
+            if (t0 == 0) t0 = t;
+            else if (t - t0 > WAIT_LIMIT_NS) { abort_pair(cx); ok = false; break; }
+          }
         }
       }
-    }
-    if (named_bar_red_or(1, GROUP, !ok)) return;
-    const bool pages_ok = !paged || request_pages_ok(p, u.b, u.nkeys);
-    const int R0 = u.mt * BM;
-    const int rows_in = rows_req - R0 < BM ? rows_req - R0 : BM;
-    const int lo = u.sp * rows_in / S, hi = (u.sp + 1) * rows_in / S;
-    const int mid = (lo + hi) / 2;
-    const int a = rank == 0 ? lo : mid, e = rank == 0 ? mid : hi;
-    for (int rr = a + wid; rr < e && pages_ok; rr += GROUP / 32) {
-      const int64_t row = (int64_t)u.b * rows_req + R0 + rr;
-      const float l0 = lane < S ? __ldcg(p.part_lse + (int64_t)lane * rows_all + row) : -INFINITY;
-      const float l1 = lane + 32 < S ? __ldcg(p.part_lse + (int64_t)(lane + 32) * rows_all + row) : -INFINITY;
-      float mx = fmaxf(l0, l1);
+      if (named_bar_red_or(1, GROUP, !ok)) return;
+      const bool pages_ok = !paged || request_pages_ok(p, b, nkeys);
+      const bool s0 = lane < S && partition_busy(T, lane, S);
+      const bool s1 = lane + 32 < S && partition_busy(T, lane + 32, S);
+      for (int64_t row = row0 + wid; row < row1 && pages_ok; row += GROUP / 32) {
+        const float l0 = s0 ? __ldcg(p.part_lse + (int64_t)lane * rows_all + row) : -INFINITY;
+        const float l1 = s1 ? __ldcg(p.part_lse + (int64_t)(lane + 32) * rows_all + row) : -INFINITY;
+        float mx = fmaxf(l0, l1);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float LOG2E = 1.4426950408889634f;
-      const float w0 = mx == -INFINITY ? 0.f : ex2((l0 - mx) * LOG2E);
-      const float w1 = mx == -INFINITY ? 0.f : ex2((l1 - mx) * LOG2E);
-      float sum = w0 + w1;
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float LOG2E = 1.4426950408889634f;
+        const float w0 = mx == -INFINITY ? 0.f : ex2((l0 - mx) * LOG2E);
+        const float w1 = mx == -INFINITY ? 0.f : ex2((l1 - mx) * LOG2E);
+        float sum = w0 + w1;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      float acc[16];
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        float acc[16];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) acc[q] = 0.f;
-      for (int s = 0; s < S; ++s) {
-        const float ws = __shfl_sync(0xffffffffu, s < 32 ? w0 : w1, s & 31);
-        if (ws == 0.f) continue;                      // empty partition (uniform over the warp)
-        const float4* src = reinterpret_cast<const float4*>(p.part_o + ((int64_t)s * rows_all + row) * KD_D_C + lane * 16);
+        for (int q = 0; q < 16; ++q) acc[q] = 0.f;
+        for (int sp = 0; sp < S; ++sp) {
+          const float ws = __shfl_sync(0xffffffffu, sp < 32 ? w0 : w1, sp & 31);
+          if (ws == 0.f) continue;                    // empty or idle partition (uniform over the warp)
+          const float4* src =
+              reinterpret_cast<const float4*>(p.part_o + ((int64_t)sp * rows_all + row) * KD_D_C + lane * 16);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 v = __ldcg(src + q);
-          acc[4 * q + 0] = fmaf(ws, v.x, acc[4 * q + 0]);
-          acc[4 * q + 1] = fmaf(ws, v.y, acc[4 * q + 1]);
-          acc[4 * q + 2] = fmaf(ws, v.z, acc[4 * q + 2]);
-          acc[4 * q + 3] = fmaf(ws, v.w, acc[4 * q + 3]);
+          for (int q = 0; q < 4; ++q) {
+            const float4 v = __ldcg(src + q);
+            acc[4 * q + 0] = fmaf(ws, v.x, acc[4 * q + 0]);
+            acc[4 * q + 1] = fmaf(ws, v.y, acc[4 * q + 1]);
+            acc[4 * q + 2] = fmaf(ws, v.z, acc[4 * q + 2]);
+            acc[4 * q + 3] = fmaf(ws, v.w, acc[4 * q + 3]);
+          }
         }
+        const float inv = sum > 0.f ? 1.f / sum : 0.f;
+        uint16_t* dst = p.out + row * KD_D_C + lane * 16;
+        st_global_v4(dst, pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                     pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+        st_global_v4(dst + 8, pack_bf16x2(acc[8] * inv, acc[9] * inv), pack_bf16x2(acc[10] * inv, acc[11] * inv),
+                     pack_bf16x2(acc[12] * inv, acc[13] * inv), pack_bf16x2(acc[14] * inv, acc[15] * inv));
+        if (lane == 0) p.lse[row] = sum > 0.f ? mx + __logf(sum) : -INFINITY;
       }
-      const float inv = sum > 0.f ? 1.f / sum : 0.f;
-      uint16_t* dst = p.out + row * KD_D_C + lane * 16;
-      st_global_v4(dst, pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                   pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
-      st_global_v4(dst + 8, pack_bf16x2(acc[8] * inv, acc[9] * inv), pack_bf16x2(acc[10] * inv, acc[11] * inv),
-                   pack_bf16x2(acc[12] * inv, acc[13] * inv), pack_bf16x2(acc[14] * inv, acc[15] * inv));
-      if (lane == 0) p.lse[row] = sum > 0.f ? mx + __logf(sum) : -INFINITY;
+      named_bar_sync(1, GROUP);
+      const int mine = (int)(row1 - row0);
+      if (tid == 0 && atomicAdd(ticket + 1, mine) + mine == rows_in) {
+        ticket[0] = 0;
+        ticket[1] = 0;
+      }
     }
-    // the last of the tile's 2 S merging CTAs returns the ticket to zero for the next launch
-    named_bar_sync(1, GROUP);
-    if (tid == 0 && atomicAdd(ticket + 1, 1) == 2 * S - 1) {
-      ticket[0] = 0;
-      ticket[1] = 0;
-    }
+    row0 = row1;
   }
 }
 
@@ -1013,6 +1113,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
     for (int i = 0; i < NBAR; ++i) {
       uint32_t cnt = 1;
       if (i == QT_FULL || i == S_EMPTY || i == CORR_DONE || i == O_FREE) cnt = GROUP;
+      if (i >= SCHED_EMPTY && i < SCHED_EMPTY + NS) cnt = SCHED_READERS;
       mbar_init(cx.bar(i), cnt);
     }
     *cx.abort_flag = 0u;
@@ -1056,24 +1157,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   bool ok = true;
   if (rank == 0) {
     if (warp == 0) {
-      qk_producer<PAGED>(cx, p, order, cid, ptab, &tm_qa, &tm_qr, &tm_c, &tm_r);
+      qk_producer<PAGED>(cx, p, order, gbase, ptab, &tm_qa, &tm_qr, &tm_c, &tm_r);
     } else if (warp == 1) {
-      if (lane == 0) qk_mma(cx, p, order, cid, tmem);
+      if (lane == 0) qk_mma(cx, p, order, gbase, tmem);
       __syncwarp();
     } else {
-      ok = qk_softmax(cx, p, order, cid, gbase, tmem);
+      ok = qk_softmax(cx, p, order, gbase, tmem);
     }
   } else {
     if (warp == 0) {
-      pv_producer<PAGED>(cx, p, order, cid, ptab, &tm_v);
+      pv_producer<PAGED>(cx, p, order, gbase, ptab, &tm_v);
     } else if (warp == 1) {
-      pv_mma(cx, p, order, cid, gbase, tmem);
+      pv_mma(cx, p, order, gbase, tmem);
     } else {
-      ok = pv_epilogue(cx, p, order, cid, gbase, tmem, PAGED);
+      ok = pv_epilogue(cx, p, order, gbase, tmem, PAGED);
     }
   }
   if (warp >= 2 && p.splits > 1 && !named_bar_red_or(1, GROUP, !ok || *cx.abort_flag))
-    merge_splits(cx, p, order, cid, rank, PAGED);
+    merge_splits(cx, p, cid, rank, PAGED);
 
   // ------------------------------------------------------- teardown
   __syncwarp();          // the roles leave lanes behind (single-lane issuers, lane 64's waits)
@@ -1172,7 +1273,9 @@ int auto_splits(int B, int n, int H, int64_t cap, int pairs) {
   return best;
 }
 
-// Workspace: 256-byte control block (int32 error word first), then, with splits:
+// Workspace: 256-byte control block (int32 error word at byte 0; the unit
+// counter and the count of clusters out of work, two uint64 at bytes 8 and 16,
+// which every launch returns to zero), then, with splits:
 // per-M-tile tickets [B * mtiles][2] int32, partial lse [S][rows] and partial
 // outputs [S][rows][512] fp32.
 struct WsLayout {
@@ -1286,6 +1389,7 @@ static int verify_attn_impl(const kd_bf16_t* q_abs, const kd_bf16_t* q_rope, con
   prm.out = out;
   prm.lse = lse;
   prm.err = reinterpret_cast<int32_t*>(ws);
+  prm.sched = reinterpret_cast<unsigned long long*>(ws + 8);
   prm.tickets = splits > 1 ? reinterpret_cast<int32_t*>(ws + wl.tickets) : nullptr;
   prm.part_lse = splits > 1 ? reinterpret_cast<float*>(ws + wl.part_lse) : nullptr;
   prm.part_o = splits > 1 ? reinterpret_cast<float*>(ws + wl.part_o) : nullptr;
