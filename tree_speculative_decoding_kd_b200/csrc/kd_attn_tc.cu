@@ -185,10 +185,19 @@ struct Ctx {
   __device__ uint32_t bar(int i) const { return base + 8u * (uint32_t)i; }
 };
 
-__device__ __noinline__ void abort_pair(Ctx cx) {
+// Gives up on the pair: both CTAs' abort flags set, KD_DEV_TIMEOUT raised, and the
+// wait that gave up recorded in the workspace's control block: the launch's first
+// at byte 4, each warp's first at byte 32 + 4 (12 rank + warp); each word is bit 31
+// set, CTA rank at bit 24, warp at bit 16, barrier index at bit 4, parity at bit 0
+// (0 while nothing gave up).
+__device__ __noinline__ void abort_pair(Ctx cx, uint32_t bar = 0u, uint32_t par = 0u) {
   *cx.abort_flag = 1u;
   st_cluster_u32(map_to_rank(cx.base + OFF_ABORT, cx.peer), 1u);
   raise_dev_error(cx.err, KD_DEV_TIMEOUT);
+  const uint32_t rank = cluster_ctarank(), warp = threadIdx.x >> 5;
+  const uint32_t site = 0x80000000u | (rank << 24) | (warp << 16) | (((bar - cx.base) >> 3) << 4) | (par & 1u);
+  atomicCAS(reinterpret_cast<unsigned int*>(cx.err + 1), 0u, site);
+  atomicCAS(reinterpret_cast<unsigned int*>(cx.err + 8 + 12 * rank + warp), 0u, site);
 }
 
 // Bounded wait for the phase of `bar` with parity `par` to complete.  With
@@ -205,7 +214,7 @@ __device__ __forceinline__ bool wait_bar(const Ctx& cx, uint32_t bar, uint32_t p
       const uint64_t t = globaltimer();
       if (t0 == 0) t0 = t;
       else if (t - t0 > WAIT_LIMIT_NS) {
-        if (!drain) abort_pair(cx);
+        if (!drain) abort_pair(cx, bar, par);
         return false;
       }
     }
@@ -1273,8 +1282,9 @@ int auto_splits(int B, int n, int H, int64_t cap, int pairs) {
   return best;
 }
 
-// Workspace: 256-byte control block (int32 error word at byte 0; the unit
-// counter and the count of clusters out of work, two uint64 at bytes 8 and 16,
+// Workspace: 256-byte control block (int32 error word at byte 0, the first wait
+// that gave up at byte 4, each warp's at bytes 32..127; the unit counter and the
+// count of clusters out of work, two uint64 at bytes 8 and 16,
 // which every launch returns to zero), then, with splits:
 // per-M-tile tickets [B * mtiles][2] int32, partial lse [S][rows] and partial
 // outputs [S][rows][512] fp32.
