@@ -58,6 +58,59 @@ def test_paged_attention_matches_contiguous_bits(kd, name, B, P, splits):
         assert ok, e
 
 
+@pytest.mark.parametrize("name,B,P,splits", [("kimi_single", None, 128, 3), ("batched", 4, 256, 1),
+                                             ("batched", 3, 64, 2)])
+def test_paged_attention_matches_oracle(kd, name, B, P, splits):
+    """The paged attention against the oracle run on the logical view of the page pool
+    (not through the contiguous kernel): multi-tile requests, split partitions merged
+    in the launch, page sizes below, at and above the 128-key tile."""
+    cfg = W.CONFIGS[name] if B is None else W.scaled(W.CONFIGS[name], B=B)
+    wl = W.make_workload(cfg)
+    st = wl.step
+    cp, rp, pt = W.to_paged(wl.c_kv, wl.k_rope, P, seed=P + 1)
+    ws = kd.new_workspace(cfg.B, cfg.n, cfg.H, pt.shape[1] * P, splits)
+    out, lse = kd.kd_tree_verify_attn_paged(kd.bf16_from_bits(st.q_abs), kd.bf16_from_bits(st.q_rope),
+                                            kd.bf16_from_bits(cp), kd.bf16_from_bits(rp), dev_i32(pt), P,
+                                            dev_i32(wl.cache_lens), masks(st), None, cfg.scale,
+                                            workspace=ws, kv_splits=splits)
+    torch.cuda.synchronize()
+    assert kd.kd_read_device_error(ws) == 0
+    vis = np.stack([oracle.visibility_words(p) for p in st.parents])
+    ro, rl = oracle.tree_verify_attention(st.q_abs, st.q_rope, oracle.cache.paged_view(cp, pt, P),
+                                          oracle.cache.paged_view(rp, pt, P), wl.cache_lens, vis, cfg.scale)
+    o = (kd.bits_from_bf16(out).astype(np.uint32) << 16).view(np.float32)
+    ok, e = attn_within_tolerance(o, lse.cpu().numpy(), ro, rl)
+    assert ok, e
+
+
+@pytest.mark.parametrize("splits", [1, 2])
+def test_paged_attention_bad_page_is_flagged_and_skipped(kd, splits):
+    """A page id outside the pool among the pages a request reads: KD_DEV_BAD_PAGE,
+    that request's outputs are left as they were, the other request is unaffected."""
+    wl = W.make_workload(W.scaled(W.CONFIGS["tiny"], B=2, L_lo=600, L_hi=700))
+    st, cfg = wl.step, wl.cfg
+    P = 64
+    cp, rp, pt = W.to_paged(wl.c_kv, wl.k_rope, P, seed=5)
+    bad = pt.copy()
+    bad[1, 3] = cp.shape[0] // P + 11                                 # a committed page of request 1
+    out = torch.full((cfg.B, cfg.n, cfg.H, 512), 3.0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((cfg.B, cfg.n, cfg.H), 5.0, dtype=torch.float32, device="cuda")
+    ws = kd.new_workspace(cfg.B, cfg.n, cfg.H, pt.shape[1] * P, splits)
+    kd.kd_tree_verify_attn_paged(kd.bf16_from_bits(st.q_abs), kd.bf16_from_bits(st.q_rope),
+                                 kd.bf16_from_bits(cp), kd.bf16_from_bits(rp), dev_i32(bad), P,
+                                 dev_i32(wl.cache_lens), masks(st), None, cfg.scale, out=out, lse=lse,
+                                 workspace=ws, kv_splits=splits)
+    torch.cuda.synchronize()
+    assert "BAD_PAGE" in kd.decode_device_error(kd.kd_read_device_error(ws))
+    assert (out[1].float() == 3.0).all() and (lse[1] == 5.0).all()
+    vis = np.stack([oracle.visibility_words(p) for p in st.parents])
+    ro, rl = oracle.tree_verify_attention(st.q_abs[:1], st.q_rope[:1], wl.c_kv[:1], wl.k_rope[:1],
+                                          wl.cache_lens[:1], vis[:1], cfg.scale)
+    o = (kd.bits_from_bf16(out[:1]).astype(np.uint32) << 16).view(np.float32)
+    ok, e = attn_within_tolerance(o, lse[:1].cpu().numpy(), ro, rl)
+    assert ok, e
+
+
 @pytest.mark.parametrize("P", [1, 16, 64])
 def test_paged_write_and_compact_bitexact(kd, P):
     wl = W.make_workload(W.scaled(W.CONFIGS["kimi_single"], B=3, L_lo=100, L_hi=300))
