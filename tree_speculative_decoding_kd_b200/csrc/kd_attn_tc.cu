@@ -247,6 +247,27 @@ __device__ __forceinline__ uint32_t mask_word(const uint32_t (&w)[4], int q) {
   return q == 0 ? w[0] : (q == 1 ? w[1] : (q == 2 ? w[2] : w[3]));
 }
 
+// Bits kt .. kt + 63 of the visibility string of one tree row, for the keys at
+// and past the first tree slot L: key L + k is visible for k < 0 (committed
+// keys), for 0 <= k < n when bit k of the row's mask is set, and never for k >= n.
+// The row's W <= 4 mask words are read from global memory.
+__device__ __noinline__ uint64_t vis_window(const uint32_t* vrow, int W, int n, int kt) {
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int lo = 32 * q;
+    const uint32_t keep = n >= lo + 32 ? ~0u : (n <= lo ? 0u : ((1u << (n - lo)) - 1u));
+    w[q] = q < W ? (vrow[q] & keep) : 0u;
+  }
+  const uint64_t a = (uint64_t)w[0] | ((uint64_t)w[1] << 32), b = (uint64_t)w[2] | ((uint64_t)w[3] << 32);
+  if (kt <= -64) return ~0ull;
+  if (kt < 0) return (a << (-kt)) | ((1ull << (-kt)) - 1ull);
+  if (kt == 0) return a;
+  if (kt < 64) return (a >> kt) | (b << (64 - kt));
+  if (kt < 128) return b >> (kt - 64);
+  return 0ull;
+}
+
 __device__ __forceinline__ float max4(float a, float b, float c, float d) {
   return fmaxf(fmaxf(a, b), fmaxf(c, d));
 }
@@ -634,21 +655,23 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
         }
         tc_fence_before();
         mbar_arrive(cx.bar(S_EMPTY));            // TMEM free for the next tile's MMAs
-        // mask: only keys at or beyond L need it
+        // mask: only keys at or beyond L need it.  The thread's 64 keys of half h
+        // are one 64-bit window of the row's visibility bits; a clear bit sets the
+        // score to -inf.  (Runs on one tile per unit, so it is kept compact: its
+        // code is cold in the instruction cache every time it runs.)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           // key index relative to the first tree slot L (fits 32 bits: keys < 2^31)
           const int kt = rel0 + t * BQ + h * BN + g * 64;
           if (kt + 64 > 0) {
-            uint32_t w[4];
+            const uint64_t vm = vis_window(vrow, W, n, kt);
+            if (vm != ~0ull) {
+              const uint32_t lo = (uint32_t)vm, hi = (uint32_t)(vm >> 32);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) w[q] = q < W ? vrow[q] : 0u;
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-              const int kk = kt + c;
-              bool vis_c = true;
-              if (kk >= 0) vis_c = (kk < n) && ((mask_word(w, kk >> 5) >> (kk & 31)) & 1u);
-              if (!vis_c) x[h][c] = -INFINITY;
+              for (int c = 0; c < 32; ++c) {
+                if (!((lo >> c) & 1u)) x[h][c] = -INFINITY;
+                if (!((hi >> c) & 1u)) x[h][c + 32] = -INFINITY;
+              }
             }
           }
         }
@@ -864,32 +887,32 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int
   __syncwarp();
 }
 
-// Each lane holds 64 bytes (16 words) of its own row; the warp moves its 32 rows
-// through its 2 KB staging slot so that every global store instruction covers 8
-// rows x 64 contiguous bytes (row r of the warp goes to dst0 + r * pitch; rows from
-// nrows on are not written).  The slot's 16-byte pieces are swizzled by row so
-// that neither the row-wise writes nor the column-wise reads conflict on banks.
-__device__ __forceinline__ void warp_store_rows(uint32_t stg, const uint32_t (&w)[16], uint8_t* dst0,
-                                                int64_t pitch, int nrows) {
+// Each lane holds 64 bytes (16 words) of its own row.  The warp writes its 32 rows
+// into its 2 KB staging slot in the 64-byte swizzled layout of the output tensor
+// map (16-byte piece c of row r at r * 64 + ((c ^ ((r >> 1) & 3)) << 4), which is
+// also free of bank conflicts), and lane 0 stores the 32-row box at (x, y, z) with
+// one TMA store; rows past the request's last row are clipped by the map.  The
+// slot is reused once the previous box has been read out of it.
+__device__ __forceinline__ void warp_store_box(uint32_t stg, const uint32_t (&w)[16], const CUtensorMap* tm,
+                                              int x, int y, int z, bool store) {
   const int lane = threadIdx.x & 31;
-  __syncwarp();                                 // the previous round's reads are done
+  if (lane == 0) bulk_wait_group_read0();
+  __syncwarp();
 #pragma unroll
   for (int c = 0; c < 4; ++c)
     st_shared_v4(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2],
                  w[4 * c + 3]);
+  fence_proxy_async_cta();
   __syncwarp();
-  const int ch = lane & 3;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int row = (lane >> 2) + 8 * j;
-    const uint4 v = ld_shared_v4(stg + row * 64 + ((ch ^ ((row >> 1) & 3)) << 4));
-    if (row < nrows) st_global_v4(dst0 + row * pitch + ch * 16, v.x, v.y, v.z, v.w);
+  if (lane == 0 && store) {
+    tma_store_3d(tm, stg, x, y, z);
+    bulk_commit_group();
   }
 }
 
 // Correction / epilogue groups: thread (g, r) owns row r, O columns [256 g, 256 g + 256).
 __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, const int* order, uint8_t* gbase,
-                                            uint32_t tmem, bool paged) {
+                                            uint32_t tmem, bool paged, const CUtensorMap* tm_o) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = (warp - 2) >> 2;
   const int quad = warp & 3;
@@ -941,39 +964,44 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
     const bool write = pages_ok && R < rows_req;
     const float inv = l > 0.f ? 1.f / l : 0.f;
     const int64_t grow = (int64_t)u.b * rows_req + R;
-    // this warp's 32 rows: the first one, and how many of them exist
+    // this warp's 32 rows start at request row R0w of plane z of the output map
+    // (request b, or partition sp of request b for split partials)
     const int R0w = u.mt * BM + quad * 32;
-    const int nrows = pages_ok ? min(max(rows_req - R0w, 0), 32) : 0;
-    const int64_t grow0 = (int64_t)u.b * rows_req + R0w;
+    const bool store = pages_ok && R0w < rows_req;
+    const int z = p.splits == 1 ? u.b : u.sp * p.B + u.b;
     const uint32_t stg = cx.base + EPI_OFF + (warp - 2) * 2048;
-    uint8_t* dst0 = p.splits == 1
-                        ? reinterpret_cast<uint8_t*>(p.out + grow0 * KD_D_C + g * 256)
-                        : reinterpret_cast<uint8_t*>(p.part_o + ((int64_t)u.sp * p.B * rows_req + grow0) * KD_D_C + g * 256);
-    for (int c = 0; c < 256 / 64; ++c) {
-      uint32_t v[64];
-      tmem_ld64(lane_addr + c * 64, v);
-      tmem_wait_ld();
-      if (c == 256 / 64 - 1) {                  // every TMEM read of this unit is done
-        tc_fence_before();
-        mbar_arrive(cx.bar(O_FREE));
+    // Rolled loops over small TMEM reads: this code runs once per unit, so its size
+    // (fetched cold every time) matters more than the exposed TMEM read latency.
+    if (p.splits == 1) {                        // bf16: eight boxes of 32 columns
+#pragma unroll 1
+      for (int c = 0; c < 256 / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(lane_addr + c * 32, v);
+        tmem_wait_ld();
+        if (c == 256 / 32 - 1) {                // every TMEM read of this unit is done
+          tc_fence_before();
+          mbar_arrive(cx.bar(O_FREE));
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          w[q] = pack_bf16x2(__uint_as_float(v[2 * q]) * inv, __uint_as_float(v[2 * q + 1]) * inv);
+        warp_store_box(stg, w, tm_o, g * 256 + c * 32, R0w, z, store);
       }
-      if (p.splits == 1) {                      // bf16: two rounds of 32 columns
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t w[16];
-#pragma unroll
-          for (int q = 0; q < 16; ++q)
-            w[q] = pack_bf16x2(__uint_as_float(v[32 * h + 2 * q]) * inv, __uint_as_float(v[32 * h + 2 * q + 1]) * inv);
-          warp_store_rows(stg, w, dst0 + (c * 64 + h * 32) * 2, KD_D_C * 2, nrows);
+    } else {                                    // fp32: sixteen boxes of 16 columns
+#pragma unroll 1
+      for (int c = 0; c < 256 / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(lane_addr + c * 16, v);
+        tmem_wait_ld();
+        if (c == 256 / 16 - 1) {
+          tc_fence_before();
+          mbar_arrive(cx.bar(O_FREE));
         }
-      } else {                                  // fp32: four rounds of 16 columns
+        uint32_t w[16];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          uint32_t w[16];
-#pragma unroll
-          for (int q = 0; q < 16; ++q) w[q] = __float_as_uint(__uint_as_float(v[16 * h + q]) * inv);
-          warp_store_rows(stg, w, dst0 + (c * 64 + h * 16) * 4, KD_D_C * 4, nrows);
-        }
+        for (int q = 0; q < 16; ++q) w[q] = __float_as_uint(__uint_as_float(v[q]) * inv);
+        warp_store_box(stg, w, tm_o, g * 256 + c * 16, R0w, z, store);
       }
     }
     if (write && g == 0) {
@@ -982,7 +1010,12 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
       else p.part_lse[(int64_t)u.sp * p.B * rows_req + grow] = lse_v;
     }
     if (p.splits > 1) {
-      // the partial is in global memory: publish it on the tile's ticket
+      // the partial is in global memory once every warp's boxes are written: publish
+      // it on the tile's ticket
+      if (lane == 0) {
+        bulk_wait_group0();
+        fence_proxy_async_global();
+      }
       named_bar_sync(1, GROUP);
       if (threadIdx.x == 64) {
         __threadfence();
@@ -991,6 +1024,8 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
     }
     ++vu;
   }
+  if (lane == 0) bulk_wait_group0();            // every box stored before the CTA leaves
+  __syncwarp();
   return ok;
 }
 
@@ -1064,19 +1099,31 @@ __device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, int
         float acc[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) acc[q] = 0.f;
-        for (int sp = 0; sp < S; ++sp) {
-          const float ws = __shfl_sync(0xffffffffu, sp < 32 ? w0 : w1, sp & 31);
-          if (ws == 0.f) continue;                    // empty or idle partition (uniform over the warp)
-          const float4* src =
-              reinterpret_cast<const float4*>(p.part_o + ((int64_t)sp * rows_all + row) * KD_D_C + lane * 16);
+        // four partitions per round, all their loads issued before any is used
+        for (int sp0 = 0; sp0 < S; sp0 += 4) {
+          float wsv[4];
+          float4 v[4][4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 v = __ldcg(src + q);
-            acc[4 * q + 0] = fmaf(ws, v.x, acc[4 * q + 0]);
-            acc[4 * q + 1] = fmaf(ws, v.y, acc[4 * q + 1]);
-            acc[4 * q + 2] = fmaf(ws, v.z, acc[4 * q + 2]);
-            acc[4 * q + 3] = fmaf(ws, v.w, acc[4 * q + 3]);
+          for (int j = 0; j < 4; ++j) {
+            const int sp = sp0 + j;
+            wsv[j] = __shfl_sync(0xffffffffu, sp < 32 ? w0 : w1, sp & 31);
+            if (sp >= S) wsv[j] = 0.f;
+            // empty or idle partitions (uniform over the warp) are not read: their
+            // partial may hold anything
+            const float4* src =
+                reinterpret_cast<const float4*>(p.part_o + ((int64_t)sp * rows_all + row) * KD_D_C + lane * 16);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) v[j][q] = wsv[j] != 0.f ? __ldcg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              acc[4 * q + 0] = fmaf(wsv[j], v[j][q].x, acc[4 * q + 0]);
+              acc[4 * q + 1] = fmaf(wsv[j], v[j][q].y, acc[4 * q + 1]);
+              acc[4 * q + 2] = fmaf(wsv[j], v[j][q].z, acc[4 * q + 2]);
+              acc[4 * q + 3] = fmaf(wsv[j], v[j][q].w, acc[4 * q + 3]);
+            }
         }
         const float inv = sum > 0.f ? 1.f / sum : 0.f;
         uint16_t* dst = p.out + row * KD_D_C + lane * 16;
@@ -1102,7 +1149,8 @@ template <bool PAGED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant__ CUtensorMap tm_qr,
                const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_r,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -1138,6 +1186,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
     tma_prefetch_desc(&tm_c);
     tma_prefetch_desc(&tm_r);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
   }
   // Longest request first: each CTA ranks the requests by cache length itself.
   const int* order = nullptr;
@@ -1179,7 +1228,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
     } else if (warp == 1) {
       pv_mma(cx, p, order, gbase, tmem);
     } else {
-      ok = pv_epilogue(cx, p, order, gbase, tmem, PAGED);
+      ok = pv_epilogue(cx, p, order, gbase, tmem, PAGED, &tm_o);
     }
   }
   if (warp >= 2 && p.splits > 1 && !named_bar_red_or(1, GROUP, !ok || *cx.abort_flag))
@@ -1223,6 +1272,26 @@ static int make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t ro
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+    return KD_ELAUNCH;
+  }
+  return KD_OK;
+}
+
+// Output map [planes][rows_req][512] (bf16 outputs, or fp32 split partials) stored in
+// 32-row boxes of 64 bytes per row, 64-byte swizzle.
+static int make_out_map(CUtensorMap* m, void* ptr, bool fp32, uint64_t rows_req, uint64_t planes) {
+  auto fn = encode_fn();
+  if (!fn) return KD_ELAUNCH;
+  const uint64_t es = fp32 ? 4 : 2;
+  cuuint64_t dims[3] = {KD_D_C, rows_req, planes};
+  cuuint64_t strides[2] = {KD_D_C * es, rows_req * KD_D_C * es};
+  cuuint32_t box[3] = {(cuuint32_t)(64 / es), 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled(out)");
     return KD_ELAUNCH;
   }
   return KD_OK;
@@ -1418,14 +1487,18 @@ static int verify_attn_impl(const kd_bf16_t* q_abs, const kd_bf16_t* q_rope, con
   prm.page_shift = paged ? (page_size == 64 ? 6 : page_size == 128 ? 7 : 8) : 0;
   prm.pages_per_req = paged ? (int)pages_per_req : 0;
   prm.num_pages = paged ? num_pages : 0;
+  CUtensorMap to;
+  if ((st = splits > 1 ? tc::make_out_map(&to, prm.part_o, true, (uint64_t)(rows / B), (uint64_t)splits * B)
+                       : tc::make_out_map(&to, out, false, (uint64_t)(rows / B), (uint64_t)B)))
+    return st;
   if (clear_ws && (st = cuda_status(cudaMemsetAsync(workspace, 0, splits > 1 ? wl.part_lse : 256, stream),
                                     "cudaMemsetAsync(workspace)")))
     return st;
   const dim3 grid((unsigned)(2 * prm.clusters));
   if (paged)
-    tc::attn_tc_kernel<true><<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(tq, tr, tcv, tkr, tv, prm);
+    tc::attn_tc_kernel<true><<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(tq, tr, tcv, tkr, tv, to, prm);
   else
-    tc::attn_tc_kernel<false><<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(tq, tr, tcv, tkr, tv, prm);
+    tc::attn_tc_kernel<false><<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(tq, tr, tcv, tkr, tv, to, prm);
   return launch_status("attn_tc_kernel");
 }
 
