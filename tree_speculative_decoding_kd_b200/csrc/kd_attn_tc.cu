@@ -167,7 +167,7 @@ struct Params {
   float* part_lse;                // [splits][B * n * H]
   int32_t* tickets;               // [B * mtiles][2]: partitions stored, merges done
   int32_t* err;
-  unsigned long long* sched;      // [0] next unit rank to hand out, [1] clusters done (self-resetting)
+  unsigned long long* sched;      // [0] ranks claimed after the first wave, [1] clusters done (self-resetting)
   int64_t cap;                    // logical slots per request (pages_per_req * P when paged)
   int64_t units;                  // B * mtiles * splits
   int B, n, H, W, mtiles, splits, clusters;
@@ -249,15 +249,16 @@ __device__ __forceinline__ uint32_t mask_word(const uint32_t (&w)[4], int q) {
 
 // Bits kt .. kt + 63 of the visibility string of one tree row, for the keys at
 // and past the first tree slot L: key L + k is visible for k < 0 (committed
-// keys), for 0 <= k < n when bit k of the row's mask is set, and never for k >= n.
-// The row's W <= 4 mask words are read from global memory.
-__device__ __noinline__ uint64_t vis_window(const uint32_t* vrow, int W, int n, int kt) {
+// keys), for 0 <= k < n when bit k of the row's mask (words m0..m3, zero past
+// W) is set, and never for k >= n.
+__device__ __noinline__ uint64_t vis_window(uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3, int n, int kt) {
+  const uint32_t mw[4] = {m0, m1, m2, m3};
   uint32_t w[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int lo = 32 * q;
     const uint32_t keep = n >= lo + 32 ? ~0u : (n <= lo ? 0u : ((1u << (n - lo)) - 1u));
-    w[q] = q < W ? (vrow[q] & keep) : 0u;
+    w[q] = mw[q] & keep;
   }
   const uint64_t a = (uint64_t)w[0] | ((uint64_t)w[1] << 32), b = (uint64_t)w[2] | ((uint64_t)w[3] << 32);
   if (kt <= -64) return ~0ull;
@@ -300,8 +301,9 @@ __device__ __forceinline__ Unit unit_at(const Params& p, const int* order, int64
 }
 
 // ---------------------------------------------------------------- schedule ring
-// Units are handed out dynamically: the QK producer claims ranks from a global
-// counter (longest requests first, see unit_at), skips those with no key tiles and
+// Units are handed out dynamically: cluster c starts with rank c, then its QK
+// producer claims ranks from a global counter (p.clusters onwards; longest requests
+// first, see unit_at), skips those with no key tiles and
 // publishes the k-th rank of its cluster in slot k % NS of a ring that both CTAs
 // hold (the peer's copy written remotely); -1 ends the cluster's work.  Every role
 // reads the ring in order and frees each slot once it has read it.
@@ -324,7 +326,7 @@ __device__ __forceinline__ int64_t claim_unit(const Params& p, const int* order,
       const Unit u = unit_at(p, order, r);
       if (u.ntiles > 0) break;
       if (!u.valid && u.mt == 0 && u.sp == 0) raise_dev_error(p.err, KD_DEV_CACHE_FULL);
-      r = (int64_t)atomicAdd(p.sched, 1ull);
+      r = (int64_t)atomicAdd(p.sched, 1ull) + p.clusters;
     }
     if (r >= p.units) r = -1;
   }
@@ -381,7 +383,37 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, cons
   const uint32_t peer_slots = map_to_rank(base + OFF_SCHED, cx.peer);
   uint32_t it = 0, uq = 0;
   bool ok = true;
-  int64_t r = claim_unit(p, order, lane == 0 ? (int64_t)atomicAdd(p.sched, 1ull) : 0);
+  // Q latent of unit u through four ring stages, then its rope chunk (whose buffer
+  // is free once every MMA of the previous unit is done)
+  auto load_q = [&](const Unit& u) -> bool {
+    const int qrow0 = u.b * p.n * p.H + u.mt * BM;
+    for (int q = 0; q < QSTAGES; ++q, ++it) {
+      const uint32_t st = it % NK;
+      if (!wait_warp(cx, cx.bar(K_EMPTY + st), ((it / NK) & 1u) ^ 1u)) return false;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(cx.bar(K_FULL + st), KCHUNK);
+        tma_load_2d(base + K_OFF + st * KCHUNK, tm_qa, 2 * q * KC, qrow0, cx.bar(K_FULL + st));
+        tma_load_2d(base + K_OFF + st * KCHUNK + CHUNK, tm_qa, (2 * q + 1) * KC, qrow0, cx.bar(K_FULL + st));
+      }
+    }
+    if (uq > 0 && !wait_warp(cx, cx.bar(Q_FREE), (uq - 1) & 1u)) return false;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(cx.bar(ROPE_FULL), CHUNK);
+      tma_load_2d(base + Q_OFF, tm_qr, 0, qrow0, cx.bar(ROPE_FULL));
+    }
+    ++uq;
+    return true;
+  };
+  // cluster c starts with unit c (no claim on the way in); later units are claimed
+  // from the counter, which hands out ranks from p.clusters on
+  int64_t r = claim_unit(p, order, (int64_t)cluster_id_x());
+  // the first unit's Q is requested before the unit is published: Q is the head of
+  // the critical path, the other roles need the unit only later
+  bool q_loaded = false;
+  if (r >= 0) {
+    if (!(ok = load_q(unit_at(p, order, r)))) r = -1;
+    q_loaded = true;
+  }
   for (int k = 0;; ++k) {
     // publish the k-th unit (or the end) once every role has read slot k - NS
     const int sl = k % NS;
@@ -396,24 +428,8 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, cons
     __syncwarp();
     if (r < 0) break;
     const Unit u = unit_at(p, order, r);
-    const int qrow0 = u.b * p.n * p.H + u.mt * BM;
-    for (int q = 0; q < QSTAGES; ++q, ++it) {
-      const uint32_t st = it % NK;
-      if (!(ok = wait_warp(cx, cx.bar(K_EMPTY + st), ((it / NK) & 1u) ^ 1u))) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(cx.bar(K_FULL + st), KCHUNK);
-        tma_load_2d(base + K_OFF + st * KCHUNK, tm_qa, 2 * q * KC, qrow0, cx.bar(K_FULL + st));
-        tma_load_2d(base + K_OFF + st * KCHUNK + CHUNK, tm_qa, (2 * q + 1) * KC, qrow0, cx.bar(K_FULL + st));
-      }
-    }
-    if (!ok) break;
-    // the rope chunk buffer is free once every MMA of the previous unit is done
-    if (uq > 0 && !(ok = wait_warp(cx, cx.bar(Q_FREE), (uq - 1) & 1u))) break;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(cx.bar(ROPE_FULL), CHUNK);
-      tma_load_2d(base + Q_OFF, tm_qr, 0, qrow0, cx.bar(ROPE_FULL));
-    }
-    ++uq;
+    if (!q_loaded && !(ok = load_q(u))) break;
+    q_loaded = false;
     const int page0 = PAGED ? (int)(u.kbeg >> p.page_shift) : 0;
     if (PAGED) {
       const int64_t kend = u.kbeg + (int64_t)u.ntiles * BQ;
@@ -432,7 +448,7 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, cons
                         ? paged_row(ptab, page0, p, u.kbeg + (int64_t)t * BQ + (i << p.page_shift)) : 0;
       }
       // claim the next unit during the last tile, so the claim's latency is hidden
-      if (t == u.ntiles - 1 && lane == 0) claimed = (int64_t)atomicAdd(p.sched, 1ull);
+      if (t == u.ntiles - 1 && lane == 0) claimed = (int64_t)atomicAdd(p.sched, 1ull) + p.clusters;
       for (int c = 0; c < NCHUNK; ++c, ++it) {
         const uint32_t st = it % NK;
         if (!(ok = wait_warp(cx, cx.bar(K_EMPTY + st), ((it / NK) & 1u) ^ 1u))) break;
@@ -638,6 +654,14 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
       }
       const int rel0 = (int)(u.kbeg - u.L);     // first key of the unit relative to slot L
       for (int t = 0; t < u.ntiles && ok; ++t, ++ts) {
+        // a tile reaching the tree slots needs the row's mask words: requested
+        // before the wait for S so that their latency hides behind it
+        uint32_t mw[4] = {0u, 0u, 0u, 0u};
+        if (rel0 + (t + 1) * BQ > 0) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (q < W) mw[q] = vrow[q];
+        }
         if (!(ok = wait_group(cx, cx.bar(S_FULL), ts & 1u))) break;
         tc_fence_after();
         // this thread's columns: keys 64 g .. 64 g + 63 of each 128-key half h of the tile
@@ -664,7 +688,7 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
           // key index relative to the first tree slot L (fits 32 bits: keys < 2^31)
           const int kt = rel0 + t * BQ + h * BN + g * 64;
           if (kt + 64 > 0) {
-            const uint64_t vm = vis_window(vrow, W, n, kt);
+            const uint64_t vm = vis_window(mw[0], mw[1], mw[2], mw[3], n, kt);
             if (vm != ~0ull) {
               const uint32_t lo = (uint32_t)vm, hi = (uint32_t)(vm >> 32);
 #pragma unroll
