@@ -98,9 +98,26 @@ int kd_tree_build_mask(const int32_t* parents, int B, int n, uint32_t* vis,
 
 /*
  * kd_verify_workspace_bytes -- workspace size for kd_tree_verify_attn with the
- * same B, n, H and kv_splits (0 = automatic).  Pure host arithmetic.  The
- * workspace must be 256-byte aligned; its first int32 is the device error word,
- * which the caller zeroes once (the library only ORs bits into it).
+ * same B, n, H, cap and kv_splits.  Returns 0 for an invalid shape.
+ *   - kv_splits = 0 sizes the split count the call itself would choose on the
+ *     CURRENT device: the automatic policy depends on how many 2-CTA clusters of
+ *     the attention kernel fit on it at once, which this function queries (and
+ *     caches per device).  With no usable device (a build host) it assumes 74
+ *     clusters, the B200 figure.  A workspace sized this way on the device that
+ *     runs the call gives the call exactly that split count; on a device that
+ *     would choose more splits the call lowers its choice to fit (see ws_bytes).
+ *   - Layout (bytes): a 256-byte control block -- int32 device error word at 0;
+ *     the first bounded wait that gave up at 4 and each warp's at 32..127 (bit 31
+ *     set, CTA rank << 24, warp << 16, barrier << 4, parity); the scheduler's two
+ *     uint64 counters at 8 and 16 -- then, with more than one split, the per-M-tile
+ *     tickets [B * ceil(n H / 128)][2] int32, the partial lse [S][B n H] fp32 and
+ *     the partial outputs [S][B n H][512] fp32, each region 256-byte aligned.
+ *   - The workspace must be 256-byte aligned and start zeroed (e.g. from
+ *     cudaMemset).  Every launch returns the counters and tickets to zero, so one
+ *     workspace serves any number of calls in stream order; the error word is only
+ *     ORed into (the caller clears it, e.g. with kd_read_device_error).  After a
+ *     KD_DEV_TIMEOUT the kernel may have stopped mid-way: zero the whole control
+ *     block and the tickets again before the next call.
  */
 size_t kd_verify_workspace_bytes(int B, int n, int H, int64_t cap, int kv_splits);
 
@@ -128,10 +145,18 @@ size_t kd_verify_workspace_bytes(int B, int n, int H, int64_t cap, int kv_splits
  *   scale           softmax scale applied to the raw dot products.
  *   out [B][n][H][512] bf16 out; lse [B][n][H] fp32 out (natural log; -inf if a
  *                   node sees no key, which cannot happen with a valid mask).
- *   workspace       >= kd_verify_workspace_bytes(B, n, H, cap, kv_splits) bytes.
- *   kv_splits       0 = automatic; otherwise the number of key-range partitions
- *                   per request (1 .. 64), combined by a log-sum-exp merge.
+ *   workspace       >= kd_verify_workspace_bytes(B, n, H, cap, kv_splits) bytes
+ *                   (ws_bytes, the caller's size), layout and lifetime as above.
+ *   kv_splits       0 = automatic: the policy's split count, lowered until its
+ *                   partials fit ws_bytes; otherwise the number of key-range
+ *                   partitions per request (1 .. 64), combined by a log-sum-exp
+ *                   merge inside the same launch.  An explicit count whose
+ *                   workspace exceeds ws_bytes returns KD_ERANGE (nothing enqueued).
  *   out/lse must not alias any input.
+ *   The work is one persistent launch of at most one 2-CTA cluster per SM pair;
+ *   units (request, 128-row M tile, key partition) are handed out longest request
+ *   first.  Every internal wait is bounded (2 s); one that gives up sets
+ *   KD_DEV_TIMEOUT and records where in the control block.
  */
 int kd_tree_verify_attn(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* q_rope,
                         const kd_bf16_t* c_kv, const kd_bf16_t* k_rope,
@@ -144,9 +169,10 @@ int kd_tree_verify_attn(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* q_rop
 /*
  * kd_tree_verify_attn_simt -- the same operation as kd_tree_verify_attn computed on
  * CUDA cores (one warp per node and head, keys streamed one at a time).  No
- * workspace, no tensor cores; a plain second GPU implementation for bring-up and
- * cross-checks.  Same arguments and checks; device errors go to `dev_error`
- * (may be NULL).
+ * workspace, no tensor cores, far slower: it is a second, independent GPU
+ * implementation that the tests use to cross-check the tensor-core kernel, not a
+ * path to serve with.  Same arguments and checks; device errors go to `dev_error`
+ * (may be NULL, in which case they are discarded).
  */
 int kd_tree_verify_attn_simt(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* q_rope,
                              const kd_bf16_t* c_kv, const kd_bf16_t* k_rope,
@@ -170,9 +196,13 @@ int kd_tree_verify_attn_simt(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* 
  *     array; an explicit kv_splits whose workspace would exceed it returns KD_ERANGE
  *     and enqueues nothing.
  *   - The call allocates nothing: no cudaMalloc/cudaFree and no allocating library
- *     routine.  It enqueues a 4-byte memset of the array's error word, the attention
- *     kernels and, when dev_error is not NULL, a 4-byte device-to-device copy of this
- *     call's KD_DEV_* bits into *dev_error (which is overwritten, not ORed).
+ *     routine.  After every argument check passed it enqueues a memset of the
+ *     array's control block (and of its split tickets, when it splits), the
+ *     attention kernel and, when dev_error is not NULL, a 4-byte device-to-device
+ *     copy of this call's KD_DEV_* bits into *dev_error (overwritten, not ORed).
+ *     With dev_error NULL this call's device errors are discarded.
+ *   - All of it is capturable into a CUDA graph (after the first call, below); a
+ *     replay re-runs the memsets, so a graph replays correctly any number of times.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) and sets kernel attributes; make that first call before
  *     any stream capture.
@@ -300,11 +330,10 @@ int kd_kv_write_nodes(kd_bf16_t* c_kv, kd_bf16_t* k_rope, int64_t kv_row_stride_
  * kd_tree_verify_attn_paged -- kd_tree_verify_attn over a paged cache.  page_size is
  * 64, 128 or 256 and pages_per_req at most 2047; the workspace is sized by
  * kd_verify_workspace_bytes(B, n, H, pages_per_req * page_size, kv_splits);
- * KD_EINVAL otherwise as the contiguous call.  This call does not check page ids:
- * the caller keeps every id a request reads in [0, num_pages) (kd_kv_write_nodes_paged
- * flags bad ids in the pages it writes).  A bad id never faults: an id below 0 or
- * from num_pages up to 2^31 / page_size reads zero rows, and a larger one wraps in
- * 32-bit row arithmetic and reads other rows of the pool.
+ * KD_EINVAL otherwise as the contiguous call.  A request whose pages
+ * [0, ceil((L + n) / page_size)) hold an id outside [0, num_pages) sets
+ * KD_DEV_BAD_PAGE and its out/lse rows are left untouched (the other requests are
+ * computed normally).  A bad id never faults: the loads use page 0 in its place.
  */
 int kd_tree_verify_attn_paged(const kd_bf16_t* q_nope_absorbed, const kd_bf16_t* q_rope,
                               const kd_bf16_t* c_pages, const kd_bf16_t* r_pages,

@@ -168,7 +168,12 @@ def kd_tree_verify_attn(q_abs, q_rope, c_kv, k_rope, cache_lens, vis, positions=
 def kd_tree_verify_attn_noalloc(q_abs, q_rope, c_kv, k_rope, cache_lens, vis, positions=None,
                                 scale=1.0 / math.sqrt(192.0), out=None, lse=None, kv_splits=0,
                                 dev_error=None, stream=None):
-    """kd_tree_verify_attn with the library's fixed workspace (no allocation by the call)."""
+    """kd_tree_verify_attn with the library's fixed workspace.
+
+    The C call allocates no device memory.  This wrapper does when `out` or `lse`
+    is None (it creates them with torch); under CUDA graph capture or on an
+    allocation-free path pass both, and `dev_error`, preallocated.  With
+    `dev_error` None the call's device errors are discarded."""
     B, n, H, sc, sr, cap, out, lse = _attn_args(q_abs, q_rope, c_kv, k_rope, cache_lens, vis,
                                                 positions, out, lse)
     _check(lib.kd_tree_verify_attn_noalloc(_ptr(q_abs), _ptr(q_rope), _ptr(c_kv), _ptr(k_rope), sc,
