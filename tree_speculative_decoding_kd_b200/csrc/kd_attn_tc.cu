@@ -121,7 +121,8 @@ enum Bar {
   PV_DRAIN = CORR_DONE + 1,             // PV: all issued PV MMAs done (before a rescale)
   SCHED_FULL = PV_DRAIN + 1,            // both: schedule slot k % NS published
   SCHED_EMPTY = SCHED_FULL + 4,         // QK: schedule slot read by all five consumers
-  NBAR = SCHED_EMPTY + 4
+  MERGE_FULL = SCHED_EMPTY + 4,         // both: a merge batch's partial rows landed (bulk copies)
+  NBAR = MERGE_FULL + 1
 };
 constexpr int NS = 4;                   // schedule ring depth
 constexpr int SCHED_READERS = 5;        // QK MMA, QK softmax, PV producer, PV MMA, PV epilogue
@@ -146,6 +147,8 @@ constexpr int P_OFF = CTRL;
 constexpr int V_OFF = P_OFF + 2 * PSLOT;
 constexpr int EPI_OFF = V_OFF + NVG * VG;                 // epilogue staging, 2 KB per worker warp
 constexpr int PV_END = EPI_OFF + 8 * 2048;
+constexpr int EPI_RING = 12;                                  // last unit: 2 KB slots per warp in P + V
+static_assert(8 * EPI_RING * 2048 <= EPI_OFF - P_OFF, "last-unit staging inside the P slots and V ring");
 constexpr int PT_OFF = QK_END > PV_END ? QK_END : PV_END;   // paged caches: the unit's page slice
 constexpr int PT_MAX = 2048;                                  // int32 entries (8 KB)
 constexpr int SMEM_BYTES = PT_OFF + PT_MAX * 4 + 1024;
@@ -284,19 +287,21 @@ struct Unit {
 // tile (the M tiles of one partition read the same keys and run side by side).
 __device__ __forceinline__ Unit unit_at(const Params& p, const int* order, int64_t r) {
   Unit u;
-  const int64_t per_req = (int64_t)p.splits * p.mtiles;
-  const int i = (int)(r / per_req);
-  const int loc = (int)(r - (int64_t)i * per_req);
+  // 32-bit divisions (64-bit ones are long subroutines): ranks stay below 2^31 and
+  // (sp + 1) * T below 64 * 2^23 since a key index fits 31 bits
+  const int per_req = p.splits * p.mtiles;
+  const int i = (int)r / per_req;
+  const int loc = (int)r - i * per_req;
   u.sp = loc / p.mtiles;
   u.mt = loc - u.sp * p.mtiles;
   u.b = order ? order[i] : i;
   u.L = p.cache_lens[u.b];
   u.valid = u.L >= 0 && u.L + p.n <= p.cap;
   u.nkeys = u.L + p.n;
-  const int64_t T = u.valid ? (u.nkeys + BQ - 1) / BQ : 0;
-  const int64_t t0 = (int64_t)u.sp * T / p.splits, t1 = (int64_t)(u.sp + 1) * T / p.splits;
-  u.ntiles = (int)(t1 - t0);
-  u.kbeg = t0 * BQ;
+  const int T = u.valid ? (int)((u.nkeys + BQ - 1) / BQ) : 0;
+  const int t0 = u.sp * T / p.splits, t1 = (u.sp + 1) * T / p.splits;
+  u.ntiles = t1 - t0;
+  u.kbeg = (int64_t)t0 * BQ;
   return u;
 }
 
@@ -912,20 +917,26 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int
 }
 
 // Each lane holds 64 bytes (16 words) of its own row.  The warp writes its 32 rows
-// into its 2 KB staging slot in the 64-byte swizzled layout of the output tensor
-// map (16-byte piece c of row r at r * 64 + ((c ^ ((r >> 1) & 3)) << 4), which is
-// also free of bank conflicts), and lane 0 stores the 32-row box at (x, y, z) with
-// one TMA store; rows past the request's last row are clipped by the map.  The
-// slot is reused once the previous box has been read out of it.
+// into a 2 KB staging slot in the 64-byte swizzled layout of the output tensor map
+// (16-byte piece c of row r at r * 64 + ((c ^ ((r >> 1) & 3)) << 4), which is also
+// free of bank conflicts); a TMA store of the 32-row box then writes it out (rows
+// past the request's last row are clipped by the map).
+__device__ __forceinline__ void stage_row(uint32_t slot, const uint32_t (&w)[16]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    st_shared_v4(slot + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2],
+                 w[4 * c + 3]);
+}
+
+// One box through the warp's single slot, reused once the previous box has been
+// read out of it.
 __device__ __forceinline__ void warp_store_box(uint32_t stg, const uint32_t (&w)[16], const CUtensorMap* tm,
                                               int x, int y, int z, bool store) {
   const int lane = threadIdx.x & 31;
   if (lane == 0) bulk_wait_group_read0();
   __syncwarp();
-#pragma unroll
-  for (int c = 0; c < 4; ++c)
-    st_shared_v4(stg + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2],
-                 w[4 * c + 3]);
+  stage_row(stg, w);
   fence_proxy_async_cta();
   __syncwarp();
   if (lane == 0 && store) {
@@ -979,6 +990,15 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
     }
     if (!ok) break;
     if (!(ok = wait_group(cx, cx.bar(STATS), vu & 1u, true) && wait_group(cx, cx.bar(O_DONE), vu & 1u))) break;
+    // The cluster's next unit (or the end) is published once this unit's loads are
+    // all issued, which O being complete implies, so this peek at the next schedule
+    // slot cannot wait on anything the epilogue still has to do.  With no next unit
+    // the P slots and the V ring are idle for good, and this unit's stores stage
+    // through them (EPI_RING slots per warp, 64 columns per round) instead of
+    // through the warp's single 2 KB slot.
+    const int kn = k + 1;
+    if (!(ok = wait_group(cx, cx.bar(SCHED_FULL + kn % NS), (kn / NS) & 1, true))) break;
+    const bool last = slots[kn % NS] < 0;
     tc_fence_after();
     const float m = fctrl[(OFF_MFIN >> 2) + r];
     const float l = fctrl[(OFF_LFIN >> 2) + r];
@@ -993,10 +1013,55 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
     const int R0w = u.mt * BM + quad * 32;
     const bool store = pages_ok && R0w < rows_req;
     const int z = p.splits == 1 ? u.b : u.sp * p.B + u.b;
-    const uint32_t stg = cx.base + EPI_OFF + (warp - 2) * 2048;
+    const uint32_t stg = last ? cx.base + P_OFF + (warp - 2) * (EPI_RING * 2048) : cx.base + EPI_OFF + (warp - 2) * 2048;
     // Rolled loops over small TMEM reads: this code runs once per unit, so its size
     // (fetched cold every time) matters more than the exposed TMEM read latency.
-    if (p.splits == 1) {                        // bf16: eight boxes of 32 columns
+    if (last) {
+      // 64 columns per round: two bf16 boxes or four fp32 boxes, one fence and one
+      // commit group per round; slots (round * boxes + j) % EPI_RING
+#pragma unroll 1
+      for (int c = 0; c < 256 / 64; ++c) {
+        uint32_t v[64];
+        tmem_ld64(lane_addr + c * 64, v);
+        tmem_wait_ld();
+        if (c == 256 / 64 - 1) {                // every TMEM read of this unit is done
+          tc_fence_before();
+          mbar_arrive(cx.bar(O_FREE));
+        }
+        // fp32 round 3 reuses round 0's slots: its boxes must be read out first
+        if (lane == 0 && p.splits > 1 && c == 3) bulk_wait_group_read<2>();
+        __syncwarp();
+        if (p.splits == 1) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            uint32_t w[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+              w[q] = pack_bf16x2(__uint_as_float(v[32 * j + 2 * q]) * inv, __uint_as_float(v[32 * j + 2 * q + 1]) * inv);
+            stage_row(stg + (2 * c + j) * 2048, w);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t w[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) w[q] = __float_as_uint(__uint_as_float(v[16 * j + q]) * inv);
+            stage_row(stg + ((4 * c + j) % EPI_RING) * 2048, w);
+          }
+        }
+        fence_proxy_async_cta();
+        __syncwarp();
+        if (lane == 0 && store) {
+          if (p.splits == 1) {
+            for (int j = 0; j < 2; ++j) tma_store_3d(tm_o, stg + (2 * c + j) * 2048, g * 256 + c * 64 + j * 32, R0w, z);
+          } else {
+            for (int j = 0; j < 4; ++j)
+              tma_store_3d(tm_o, stg + ((4 * c + j) % EPI_RING) * 2048, g * 256 + c * 64 + j * 16, R0w, z);
+          }
+          bulk_commit_group();
+        }
+      }
+    } else if (p.splits == 1) {                 // bf16: eight boxes of 32 columns
 #pragma unroll 1
       for (int c = 0; c < 256 / 32; ++c) {
         uint32_t v[32];
@@ -1056,40 +1121,58 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
 // ====================================================================== split-KV merge
 // Partition sp of request b covers QK tiles [sp T / S, (sp+1) T / S) of its T tiles;
 // partitions without tiles are never scheduled and store nothing.
-__device__ __forceinline__ bool partition_busy(int64_t T, int sp, int S) {
-  return (int64_t)(sp + 1) * T / S > (int64_t)sp * T / S;
+__device__ __forceinline__ bool partition_busy(int T, int sp, int S) {
+  return (sp + 1) * T / S > sp * T / S;
 }
 
 // After its last unit, each CTA merges a fixed share of all rows (cluster c takes
 // rows [c R / G, (c+1) R / G) of the R = B n H rows, split between its two CTAs),
-// one M tile at a time once that tile's ticket shows every busy partition stored,
-// one warp per row and 16 latent columns per lane:
+// one M tile at a time once that tile's ticket shows every busy partition stored:
 //   LSE = ln sum_s exp(lse_s),   out = sum_s exp(lse_s - LSE) o_s.
+// The partial rows of a batch of rows are brought into shared memory by bulk copies
+// all in flight at once (the P staging area and the K / V ring, idle by now: every
+// load into them has landed and every MMA reading them is done), so a batch costs
+// one memory round trip; each warp then merges rows from shared memory, lane l
+// owning the 16-byte column pieces l, l + 32, l + 64, l + 96 of the 512-wide row.
 // The merged-row count on the tile's second ticket word tells the last merger to
 // return both words to zero for the next launch.
+constexpr int MBUF_BYTES = 2 * PSLOT + NK * KCHUNK;        // STG + K ring (QK), P + V ring (PV)
+constexpr int MBUF_ROWS = MBUF_BYTES / (KD_D_C * 4);       // partial rows the buffer holds
+static_assert(2 * PSLOT + NVG * VG == MBUF_BYTES && STG_OFF + 2 * PSLOT == K_OFF && P_OFF + 2 * PSLOT == V_OFF,
+              "merge buffer: one contiguous region in both CTAs");
+
 __device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, int cid, uint32_t rank,
                                              bool paged) {
   const int tid = threadIdx.x - 64;
   const int wid = tid >> 5, lane = threadIdx.x & 31;
   const int rows_req = p.n * p.H, S = p.splits;
-  const int64_t rows_all = (int64_t)p.B * rows_req;
-  const int64_t lo = (int64_t)cid * rows_all / p.clusters, hi = (int64_t)(cid + 1) * rows_all / p.clusters;
-  const int64_t mid = (lo + hi) / 2;
-  const int64_t a = rank == 0 ? lo : mid, e = rank == 0 ? mid : hi;
-  for (int64_t row0 = a; row0 < e;) {
-    const int b = (int)(row0 / rows_req);
-    const int R0 = (int)(row0 - (int64_t)b * rows_req);
+  // 32-bit row arithmetic (B n H < 2^31): cluster c's share is q or q + 1 rows
+  const int rows_all = p.B * rows_req;
+  const int q_rows = rows_all / p.clusters, r_rows = rows_all - q_rows * p.clusters;
+  const int lo = cid * q_rows + min(cid, r_rows), hi = lo + q_rows + (cid < r_rows ? 1 : 0);
+  const int mid = (lo + hi) / 2;
+  const int a = rank == 0 ? lo : mid, e = rank == 0 ? mid : hi;
+  const uint32_t mbuf = cx.base + (rank == 0 ? STG_OFF : P_OFF);
+  const int batch_rows = MBUF_ROWS / S;                      // S <= 64 < MBUF_ROWS
+  uint32_t mph = 0;
+  for (int row0 = a; row0 < e;) {
+    const int b = row0 / rows_req;
+    const int R0 = row0 - b * rows_req;
     const int mt = R0 / BM;
     const int rows_in = rows_req - mt * BM < BM ? rows_req - mt * BM : BM;
-    const int64_t tile_end_g = (int64_t)b * rows_req + mt * BM + rows_in;
-    const int64_t row1 = tile_end_g < e ? tile_end_g : e;
+    const int tile_end_g = b * rows_req + mt * BM + rows_in;
+    const int row1 = tile_end_g < e ? tile_end_g : e;
     const int64_t L = p.cache_lens[b];
     const bool valid = L >= 0 && L + p.n <= p.cap;
     if (valid) {
       const int64_t nkeys = L + p.n;
-      const int64_t T = (nkeys + BQ - 1) / BQ;
-      int busy = 0;
-      for (int s = 0; s < S; ++s) busy += partition_busy(T, s, S);
+      const int T = (int)((nkeys + BQ - 1) / BQ);
+      // busy partitions as a bit mask (lane l decides partitions l and l + 32)
+      const bool s0 = lane < S && partition_busy(T, lane, S);
+      const bool s1 = lane + 32 < S && partition_busy(T, lane + 32, S);
+      const uint64_t busy_mask = (uint64_t)__ballot_sync(0xffffffffu, s0) |
+                                 ((uint64_t)__ballot_sync(0xffffffffu, s1) << 32);
+      const int busy = __popcll(busy_mask);
       int32_t* ticket = p.tickets + 2 * ((int64_t)b * p.mtiles + mt);
       // wait until every busy partition of the tile has stored its partial
       bool ok = true;
@@ -1106,58 +1189,80 @@ __device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, int
       }
       if (named_bar_red_or(1, GROUP, !ok)) return;
       const bool pages_ok = !paged || request_pages_ok(p, b, nkeys);
-      const bool s0 = lane < S && partition_busy(T, lane, S);
-      const bool s1 = lane + 32 < S && partition_busy(T, lane + 32, S);
-      for (int64_t row = row0 + wid; row < row1 && pages_ok; row += GROUP / 32) {
-        const float l0 = s0 ? __ldcg(p.part_lse + (int64_t)lane * rows_all + row) : -INFINITY;
-        const float l1 = s1 ? __ldcg(p.part_lse + (int64_t)(lane + 32) * rows_all + row) : -INFINITY;
-        float mx = fmaxf(l0, l1);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float LOG2E = 1.4426950408889634f;
-        const float w0 = mx == -INFINITY ? 0.f : ex2((l0 - mx) * LOG2E);
-        const float w1 = mx == -INFINITY ? 0.f : ex2((l1 - mx) * LOG2E);
-        float sum = w0 + w1;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        float acc[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) acc[q] = 0.f;
-        // four partitions per round, all their loads issued before any is used
-        for (int sp0 = 0; sp0 < S; sp0 += 4) {
-          float wsv[4];
-          float4 v[4][4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int sp = sp0 + j;
-            wsv[j] = __shfl_sync(0xffffffffu, sp < 32 ? w0 : w1, sp & 31);
-            if (sp >= S) wsv[j] = 0.f;
-            // empty or idle partitions (uniform over the warp) are not read: their
-            // partial may hold anything
-            const float4* src =
-                reinterpret_cast<const float4*>(p.part_o + ((int64_t)sp * rows_all + row) * KD_D_C + lane * 16);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) v[j][q] = wsv[j] != 0.f ? __ldcg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int bs = row0; bs < row1 && pages_ok; bs += batch_rows) {
+        const int nb = row1 - bs < batch_rows ? row1 - bs : batch_rows;
+        // slot (r, sp) of the buffer holds partial sp of row bs + r (busy partitions only)
+        if (wid == 0) {
+          if (lane == 0) mbar_arrive_expect_tx(cx.bar(MERGE_FULL), (uint32_t)(nb * busy) * (KD_D_C * 4));
+          fence_proxy_async_global();             // the partials (acquired above) feed async copies
+          __syncwarp();
+          for (int i = lane; i < nb * S; i += 32) {
+            const int r = i / S, sp = i - r * S;
+            if ((busy_mask >> sp) & 1ull)
+              bulk_load_global(mbuf + (uint32_t)i * (KD_D_C * 4),
+                               p.part_o + ((int64_t)sp * rows_all + (bs + r)) * KD_D_C, KD_D_C * 4,
+                               cx.bar(MERGE_FULL));
           }
+        }
+        // this warp's rows of the batch: the lse of its first two rows are requested
+        // before the wait, so that their latency hides behind the copies'
+        const int rw = wid;
+        float l0 = -INFINITY, l1 = -INFINITY, l0n = -INFINITY, l1n = -INFINITY;
+        if (rw < nb) {
+          if (s0) l0 = __ldcg(p.part_lse + (int64_t)lane * rows_all + (bs + rw));
+          if (s1) l1 = __ldcg(p.part_lse + (int64_t)(lane + 32) * rows_all + (bs + rw));
+        }
+        if (rw + GROUP / 32 < nb) {
+          if (s0) l0n = __ldcg(p.part_lse + (int64_t)lane * rows_all + (bs + rw + GROUP / 32));
+          if (s1) l1n = __ldcg(p.part_lse + (int64_t)(lane + 32) * rows_all + (bs + rw + GROUP / 32));
+        }
+        const bool landed = wait_bar(cx, cx.bar(MERGE_FULL), mph & 1u, false, true);
+        ++mph;
+        if (named_bar_red_or(1, GROUP, !landed)) { abort_pair(cx); return; }
+        for (int r = rw; r < nb; r += GROUP / 32) {
+          const int grow = bs + r;
+          if (r == rw + GROUP / 32) {
+            l0 = l0n;
+            l1 = l1n;
+          } else if (r != rw) {
+            l0 = s0 ? __ldcg(p.part_lse + (int64_t)lane * rows_all + grow) : -INFINITY;
+            l1 = s1 ? __ldcg(p.part_lse + (int64_t)(lane + 32) * rows_all + grow) : -INFINITY;
+          }
+          float mx = fmaxf(l0, l1);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const float LOG2E = 1.4426950408889634f;
+          const float w0 = mx == -INFINITY ? 0.f : ex2((l0 - mx) * LOG2E);
+          const float w1 = mx == -INFINITY ? 0.f : ex2((l1 - mx) * LOG2E);
+          float sum = w0 + w1;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          float acc[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) acc[q] = 0.f;
+          for (int sp = 0; sp < S; ++sp) {
+            const float ws = __shfl_sync(0xffffffffu, sp < 32 ? w0 : w1, sp & 31);
+            if (ws == 0.f) continue;              // empty or idle partition (uniform over the warp)
+            const uint32_t src = mbuf + (uint32_t)(r * S + sp) * (KD_D_C * 4) + lane * 16;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              acc[4 * q + 0] = fmaf(wsv[j], v[j][q].x, acc[4 * q + 0]);
-              acc[4 * q + 1] = fmaf(wsv[j], v[j][q].y, acc[4 * q + 1]);
-              acc[4 * q + 2] = fmaf(wsv[j], v[j][q].z, acc[4 * q + 2]);
-              acc[4 * q + 3] = fmaf(wsv[j], v[j][q].w, acc[4 * q + 3]);
+              const uint4 v = ld_shared_v4(src + q * 512);
+              acc[4 * q + 0] = fmaf(ws, __uint_as_float(v.x), acc[4 * q + 0]);
+              acc[4 * q + 1] = fmaf(ws, __uint_as_float(v.y), acc[4 * q + 1]);
+              acc[4 * q + 2] = fmaf(ws, __uint_as_float(v.z), acc[4 * q + 2]);
+              acc[4 * q + 3] = fmaf(ws, __uint_as_float(v.w), acc[4 * q + 3]);
             }
+          }
+          const float inv = sum > 0.f ? 1.f / sum : 0.f;
+          uint16_t* dst = p.out + (int64_t)grow * KD_D_C + lane * 4;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            st_global_v2(dst + q * 128, pack_bf16x2(acc[4 * q] * inv, acc[4 * q + 1] * inv),
+                         pack_bf16x2(acc[4 * q + 2] * inv, acc[4 * q + 3] * inv));
+          if (lane == 0) p.lse[grow] = sum > 0.f ? mx + __logf(sum) : -INFINITY;
         }
-        const float inv = sum > 0.f ? 1.f / sum : 0.f;
-        uint16_t* dst = p.out + row * KD_D_C + lane * 16;
-        st_global_v4(dst, pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                     pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
-        st_global_v4(dst + 8, pack_bf16x2(acc[8] * inv, acc[9] * inv), pack_bf16x2(acc[10] * inv, acc[11] * inv),
-                     pack_bf16x2(acc[12] * inv, acc[13] * inv), pack_bf16x2(acc[14] * inv, acc[15] * inv));
-        if (lane == 0) p.lse[row] = sum > 0.f ? mx + __logf(sum) : -INFINITY;
+        named_bar_sync(1, GROUP);               // the buffer is read out before the next batch
       }
-      named_bar_sync(1, GROUP);
       const int mine = (int)(row1 - row0);
       if (tid == 0 && atomicAdd(ticket + 1, mine) + mine == rows_in) {
         ticket[0] = 0;
@@ -1504,6 +1609,7 @@ static int verify_attn_impl(const kd_bf16_t* q_abs, const kd_bf16_t* q_rope, con
   prm.mtiles = (int)((rows / B + tc::BM - 1) / tc::BM);
   prm.splits = splits;
   prm.units = (int64_t)B * prm.mtiles * splits;
+  if (prm.units > INT32_MAX) return KD_EINVAL;     // unit ranks are 32-bit on the device
   prm.clusters = (int)(prm.units < pairs ? prm.units : pairs);
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.page_table = page_table;
