@@ -469,3 +469,23 @@ def test_loop_full_size_two_steps(kd):
         assert np.array_equal(host_u16(kd, ck), c_np)
         assert np.array_equal(host_u16(kd, kr), r_np)
     assert kd.kd_read_device_error(err) == 0 and kd.kd_read_device_error(ws) == 0
+
+
+@pytest.mark.parametrize("name,kw,splits,mul", [("kimi_single", {}, 0, 1.0), ("batched", {"B": 8}, 0, 1.0),
+                                                ("batched", {"B": 3}, 3, 1.0),
+                                                ("batched", {"B": 4, "L_lo": 700, "L_hi": 2000}, 2, 32.0)])
+def test_attn_repeatable_bits(kd, name, kw, splits, mul):
+    """The attention's arithmetic order is fixed (units, tiles, the P hand-over, the
+    rescales and the split merge), so repeated calls give the same bits; a race in any
+    hand-over between the two CTAs or across clusters would show as a difference."""
+    wl = W.make_workload(small(name, **kw) if kw else W.CONFIGS[name])
+    scale = wl.cfg.scale * mul
+    first = run_attn(kd, wl, kv_splits=splits, scale=scale)
+    assert first[2] == 0
+    for _ in range(4):
+        again = run_attn(kd, wl, kv_splits=splits, scale=scale)
+        assert again[2] == 0
+        assert np.array_equal(again[0].view(np.uint32), first[0].view(np.uint32))
+        assert np.array_equal(again[1].view(np.uint32), first[1].view(np.uint32))
+    ro, rl = oracle_attn(wl, scale=scale)
+    assert_attn(first[0], first[1], ro, rl, f"{name} x{mul}")
