@@ -1,6 +1,10 @@
 """Builds libkdverify.so in-tree for sm_100a with nvcc (no JIT cache).
 
-    python -m tree_speculative_decoding_kd_b200.build
+    python -m tree_speculative_decoding_kd_b200.build           # the library
+    python -m tree_speculative_decoding_kd_b200.build --trace   # + libkdverify_trace.so
+
+The trace build compiles the attention with -DKD_TRACE: the same kernel recording a
+per-CTA timeline and wait counters of each launch (read by trace.py).
 """
 from __future__ import annotations
 
@@ -16,6 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libkdverify.so")
+TRACE_LIB = os.path.join(PKG, "libkdverify_trace.so")
 
 SOURCES = ["kd_tree.cu", "kd_attn_simt.cu", "kd_attn_tc.cu", "kd_argmax.cu", "kd_tree_build.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -30,9 +35,9 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(OBJ, os.path.splitext(src)[0] + ".o")
-    cmd = [nvcc(), *ARCH, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+def _compile(src: str, verbose: bool, extra=(), suffix: str = "") -> str:
+    obj = os.path.join(OBJ, os.path.splitext(src)[0] + suffix + ".o")
+    cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", os.path.join(CSRC, src), "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -62,5 +67,21 @@ def build(verbose: bool = False, force: bool = False) -> str:
     return LIB
 
 
+def build_trace(verbose: bool = False) -> str:
+    """libkdverify_trace.so: the library with the attention compiled with -DKD_TRACE."""
+    build(verbose)
+    objs = [os.path.join(OBJ, os.path.splitext(s)[0] + ".o") for s in SOURCES if s != "kd_attn_tc.cu"]
+    objs.append(_compile("kd_attn_tc.cu", verbose, ["-DKD_TRACE"], "_trace"))
+    tmp = TRACE_LIB + ".tmp"
+    r = subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static"], capture_output=True,
+                       text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+    os.replace(tmp, TRACE_LIB)
+    return TRACE_LIB
+
+
 if __name__ == "__main__":
     print(build(verbose="-v" in sys.argv, force=True))
+    if "--trace" in sys.argv:
+        print(build_trace(verbose="-v" in sys.argv))

@@ -71,6 +71,32 @@ namespace tc {
 
 using namespace ptx;
 
+// ---------------------------------------------------------------- trace build
+// Built with -DKD_TRACE (libkdverify_trace.so, "python -m
+// tree_speculative_decoding_kd_b200.build --trace"), the kernel records, per CTA,
+// the global timer at fixed points of each role (slots 0..31) and cycle counters
+// of the main waits (slots 32..63); tree_speculative_decoding_kd_b200/trace.py names
+// the slots and prints a launch's timeline.  The product library has none of it.
+// Counters live in registers of the role's thread and reach memory once, when the
+// role ends, so that they barely disturb what they measure.
+#ifdef KD_TRACE
+constexpr int TRACE_CTAS = 160, TRACE_SLOTS = 64;
+__device__ unsigned long long g_trace[TRACE_CTAS][TRACE_SLOTS];
+#define KD_EV(i) (g_trace[blockIdx.x][(i)] = globaltimer())
+#define KD_CTR(c) long long c = 0
+#define KD_T0(t) const long long t = clock64()
+#define KD_ADD(c, t) ((c) += clock64() - (t))
+#define KD_INC(c) (++(c))
+#define KD_FLUSH(i, c) atomicAdd(&g_trace[blockIdx.x][(i)], (unsigned long long)(c))
+#else
+#define KD_EV(i) ((void)0)
+#define KD_CTR(c) ((void)0)
+#define KD_T0(t) ((void)0)
+#define KD_ADD(c, t) ((void)0)
+#define KD_INC(c) ((void)0)
+#define KD_FLUSH(i, c) ((void)0)
+#endif
+
 constexpr int NTHREADS = 320;           // warp 0 TMA, warp 1 MMA, warps 2..9 two 4-warp groups
 constexpr int GROUP = 256;              // threads of the two 4-warp groups
 constexpr int BM = 128;                 // query rows per M tile
@@ -412,11 +438,13 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, cons
   // cluster c starts with unit c (no claim on the way in); later units are claimed
   // from the counter, which hands out ranks from p.clusters on
   int64_t r = claim_unit(p, order, (int64_t)cluster_id_x());
+  if (lane == 0) KD_EV(4);
   // the first unit's Q is requested before the unit is published: Q is the head of
   // the critical path, the other roles need the unit only later
   bool q_loaded = false;
   if (r >= 0) {
     if (!(ok = load_q(unit_at(p, order, r)))) r = -1;
+    if (lane == 0) KD_EV(5);
     q_loaded = true;
   }
   for (int k = 0;; ++k) {
@@ -430,6 +458,7 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, cons
       mbar_arrive(cx.bar(SCHED_FULL + sl));
       mbar_arrive_remote(map_to_rank(cx.bar(SCHED_FULL + sl), cx.peer));
     }
+    if (lane == 0 && k == 0) KD_EV(6);
     __syncwarp();
     if (r < 0) break;
     const Unit u = unit_at(p, order, r);
@@ -474,6 +503,7 @@ __device__ __forceinline__ void qk_producer(const Ctx& cx, const Params& p, cons
       }
     }
     if (!ok) break;
+    if (lane == 0) KD_EV(7);
     r = claim_unit(p, order, claimed);
   }
   // every armed copy must land before the CTA may leave (bounded, even after an abort)
@@ -498,22 +528,42 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, const Params& p, const int
   volatile int64_t* slots = sched_slots(gbase);
   uint32_t it = 0, ts = 0, uq = 0;
   bool ok = true;
+  KD_CTR(c_se);
+  KD_CTR(c_kf);
+  KD_CTR(c_is);
+  KD_CTR(c_nt);
+  KD_CTR(c_us);
+  KD_CTR(c_qt);
+  KD_CTR(c_nu);
   for (int k = 0; ok; ++k) {
     if (!(ok = wait_bar(cx, cx.bar(SCHED_FULL + k % NS), (k / NS) & 1, true))) break;
     const int64_t r = slots[k % NS];
     sched_release(cx, k % NS, false);
     if (r < 0) break;
+    KD_T0(tu);
     const Unit u = unit_at(p, order, r);
     it += QSTAGES;                              // Q stages are consumed by the softmax groups
+    KD_T0(tq);
     if (!(ok = wait_bar(cx, cx.bar(QT_FULL), uq & 1u) && wait_bar(cx, cx.bar(ROPE_FULL), uq & 1u))) break;
+    KD_ADD(c_qt, tq);
+    KD_ADD(c_us, tu);
+    KD_INC(c_nu);
+    if (uq == 0) KD_EV(8);
     tc_fence_after();
     for (int t = 0; t < u.ntiles && ok; ++t, ++ts) {
+      KD_T0(te);
       if (!(ok = wait_bar(cx, cx.bar(S_EMPTY), (ts & 1u) ^ 1u))) break;
+      KD_ADD(c_se, te);
+      KD_INC(c_nt);
       tc_fence_after();
       const uint32_t d = tmem + TS;
       for (int c = 0; c < NCHUNK; ++c, ++it) {
         const uint32_t st = it % NK;
+        KD_T0(tk);
         if (!(ok = wait_bar(cx, cx.bar(K_FULL + st), (it / NK) & 1u))) break;
+        KD_ADD(c_kf, tk);
+        if (ts == 0 && c == 0) KD_EV(9);
+        KD_T0(ti);
         tc_fence_after();
         const uint32_t b0 = base + K_OFF + st * KCHUNK;
         if (c < NQT) {
@@ -526,12 +576,22 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, const Params& p, const int
             mma_bf16_ss(d, desc_k(base + Q_OFF + kk * 32), desc_k(b0 + kk * 32), IDESC_QK, 1u);
         }
         tc_commit(cx.bar(K_EMPTY + st));
+        KD_ADD(c_is, ti);
       }
       if (ok) tc_commit(cx.bar(S_FULL));
+      if (ts == 0) KD_EV(10);
+      KD_EV(11);
     }
     if (ok) tc_commit(cx.bar(Q_FREE));
     ++uq;
   }
+  KD_FLUSH(32, c_se);
+  KD_FLUSH(33, c_kf);
+  KD_FLUSH(34, c_is);
+  KD_FLUSH(35, c_nt);
+  KD_FLUSH(36, c_us);
+  KD_FLUSH(37, c_qt);
+  KD_FLUSH(38, c_nu);
   tc_commit(cx.bar(DRAIN));
   wait_bar(cx, cx.bar(DRAIN), 0, false, true);
 }
@@ -628,8 +688,12 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
 
   volatile int64_t* slots = sched_slots(gbase);
   uint32_t pos = 0, ts = 0, pc = 0, nq = 0, ns = 0;
+  KD_CTR(c_sf);
+  KD_CTR(c_em);
+  KD_CTR(c_tt);
   bool ok = wait_group(cx, cx.bar(SCHED_FULL), 0, true);
   if (ok && slots[0] >= 0) ok = copy_q(cx, gbase, lane_addr, 0, g, r);     // the first unit's Q
+  if (threadIdx.x == 64) KD_EV(12);
   for (int k = 0; ok; ++k) {
     if (!(ok = wait_group(cx, cx.bar(SCHED_FULL + k % NS), (k / NS) & 1, true))) break;
     const int64_t rk = slots[k % NS];
@@ -667,7 +731,10 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
           for (int q = 0; q < 4; ++q)
             if (q < W) mw[q] = vrow[q];
         }
+        KD_T0(tsf);
         if (!(ok = wait_group(cx, cx.bar(S_FULL), ts & 1u))) break;
+        KD_ADD(c_sf, tsf);
+        if (threadIdx.x == 64) KD_EV(15);
         tc_fence_after();
         // this thread's columns: keys 64 g .. 64 g + 63 of each 128-key half h of the tile
         float x[2][64];
@@ -684,6 +751,7 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
         }
         tc_fence_before();
         mbar_arrive(cx.bar(S_EMPTY));            // TMEM free for the next tile's MMAs
+        if (threadIdx.x == 64 && ts == 0) KD_EV(13);
         // mask: only keys at or beyond L need it.  The thread's 64 keys of half h
         // are one 64-bit window of the row's visibility bits; a clear bit sets the
         // score to -inf.  (Runs on one tile per unit, so it is kept compact: its
@@ -704,6 +772,7 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
             }
           }
         }
+        if (threadIdx.x == 64) KD_EV(16);
         // row max of the raw scores (the scale is positive, so it commutes with max)
         float mx[4] = {x[0][0], x[0][1], x[0][2], x[0][3]};
 #pragma unroll
@@ -732,6 +801,7 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
           m_ref = tmax;
         }
         const float mb = m_ref == -INFINITY ? 0.f : m_ref;
+        KD_T0(tem);
         ok = emit_p(cx, gbase, x[0], pc, p.scale_log2, mb, alpha, rescale_row, r, g, peer_p, peer_ctrl,
                     l_part);
         if (ok && t == u.ntiles - 1) {
@@ -747,6 +817,12 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
         ok = ok && emit_p(cx, gbase, x[1], pc + 1, p.scale_log2, mb, 1.f, false, r, g, peer_p, peer_ctrl,
                           l_part);
         pc += 2;
+        KD_ADD(c_em, tem);
+        KD_ADD(c_tt, tsf);
+        if (threadIdx.x == 64) {
+          if (ts == 0) KD_EV(14);
+          KD_EV(17);
+        }
       }
       if (!ok) break;
       pos += QSTAGES + NCHUNK * (uint32_t)u.ntiles;
@@ -765,7 +841,13 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
     }
     named_bar_sync(1, GROUP);
     if (threadIdx.x == 64) mbar_arrive_remote(peer_ctrl + 8u * STATS);
+    if (threadIdx.x == 64) KD_EV(18);
     ++ns;
+  }
+  if (threadIdx.x == 64) {
+    KD_FLUSH(40, c_sf);
+    KD_FLUSH(41, c_em);
+    KD_FLUSH(42, c_tt);
   }
   // the peer's last arrivals on this CTA's barriers (P slots freed, statistics
   // read) must land before the CTA leaves
@@ -819,6 +901,7 @@ __device__ __forceinline__ void pv_producer(const Ctx& cx, const Params& p, cons
             for (int q = 0; q < 4; ++q)
               tma_load_2d(cx.base + V_OFF + gs * VG + q * VCH, tm_v, (hh * 4 + q) * KC, krow,
                           cx.bar(V_FULL + gs));
+            if (gi == 0) KD_EV(19);
           }
         }
       }
@@ -837,6 +920,9 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int
   volatile int64_t* slots = sched_slots(gbase);
   bool ok = true;
   uint32_t gi = 0, pc = 0, vu = 0, nres = 0, nd = 0;
+  KD_CTR(c_pf);
+  KD_CTR(c_vf);
+  KD_CTR(c_nh);
   for (int k = 0; ok; ++k) {
     if (!(ok = wait_warp(cx, cx.bar(SCHED_FULL + k % NS), (k / NS) & 1, true))) break;
     const int64_t r = slots[k % NS];
@@ -849,7 +935,11 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int
     for (int t = 0; t < 2 * u.ntiles && ok; ++t, ++pc) {      // P tiles of 128 keys
       const uint32_t sb = pc & 1;
       if (lane == 0) mbar_arrive_expect_tx(cx.bar(P_FULL + sb), SLOT_COPY);
+      KD_T0(tp);
       if (!(ok = wait_warp(cx, cx.bar(P_FULL + sb), (pc >> 1) & 1, true))) break;
+      KD_ADD(c_pf, tp);
+      KD_INC(c_nh);
+      if (lane == 0 && pc == 0) KD_EV(20);
       const uint32_t flag =
           *reinterpret_cast<volatile uint32_t*>(gbase + P_OFF + sb * PSLOT + SLOT_FLAG);
       if (flag && t > 0) {
@@ -871,7 +961,9 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int
         if (nv == 0) continue;             // P is zero there: nothing to add (and nothing loaded)
         for (int hh = 0; hh < 2 && ok; ++hh, ++gi) {
           const uint32_t gs = gi % NVG;
+          KD_T0(tv);
           if (!(ok = wait_warp(cx, cx.bar(V_FULL + gs), (gi / NVG) & 1u))) break;
+          KD_ADD(c_vf, tv);
           if (nv < VKEYS) {
             // rows past the request's last key may hold anything (even NaN bit
             // patterns); P is 0 there but 0 * NaN is not, so clear them.  A key row is
@@ -903,6 +995,7 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int
     if (!ok) break;
     if (lane == 0) {
       tc_commit(cx.bar(O_DONE));
+      KD_EV(21);
       ctrl[OFF_EVTYPE >> 2] = 2u;
       mbar_arrive(cx.bar(EVENT));
     }
@@ -910,6 +1003,9 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int
     ++vu;
   }
   if (lane == 0) {
+    KD_FLUSH(44, c_pf);
+    KD_FLUSH(45, c_vf);
+    KD_FLUSH(46, c_nh);
     tc_commit(cx.bar(PV_DRAIN));
     wait_bar(cx, cx.bar(PV_DRAIN), nd & 1u, false, true);
   }
@@ -990,6 +1086,7 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
     }
     if (!ok) break;
     if (!(ok = wait_group(cx, cx.bar(STATS), vu & 1u, true) && wait_group(cx, cx.bar(O_DONE), vu & 1u))) break;
+    if (threadIdx.x == 64) KD_EV(22);
     // The cluster's next unit (or the end) is published once this unit's loads are
     // all issued, which O being complete implies, so this peek at the next schedule
     // slot cannot wait on anything the epilogue still has to do.  With no next unit
@@ -1024,6 +1121,7 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
         uint32_t v[64];
         tmem_ld64(lane_addr + c * 64, v);
         tmem_wait_ld();
+        if (c == 0 && threadIdx.x == 64) KD_EV(23);
         if (c == 256 / 64 - 1) {                // every TMEM read of this unit is done
           tc_fence_before();
           mbar_arrive(cx.bar(O_FREE));
@@ -1111,6 +1209,7 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
         atom_add_release_gpu(p.tickets + 2 * ((int64_t)u.b * p.mtiles + u.mt), 1);
       }
     }
+    if (threadIdx.x == 64) KD_EV(24);
     ++vu;
   }
   if (lane == 0) bulk_wait_group0();            // every box stored before the CTA leaves
@@ -1188,6 +1287,9 @@ __device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, int
         }
       }
       if (named_bar_red_or(1, GROUP, !ok)) return;
+#ifdef KD_TRACE
+      if (threadIdx.x == 64 && g_trace[blockIdx.x][26] == 0) KD_EV(26);
+#endif
       const bool pages_ok = !paged || request_pages_ok(p, b, nkeys);
       for (int bs = row0; bs < row1 && pages_ok; bs += batch_rows) {
         const int nb = row1 - bs < batch_rows ? row1 - bs : batch_rows;
@@ -1288,6 +1390,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   const uint32_t rank = cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cid = (int)cluster_id_x();
+  if (threadIdx.x == 0) KD_EV(0);
 
   Ctx cx;
   cx.base = base;
@@ -1340,6 +1443,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + OFF_TMEM);
   int32_t* ptab = reinterpret_cast<int32_t*>(gbase + PT_OFF);
+  if (threadIdx.x == 0) KD_EV(1);
 
   bool ok = true;
   if (rank == 0) {
@@ -1360,16 +1464,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qa, const __grid_constant_
       ok = pv_epilogue(cx, p, order, gbase, tmem, PAGED, &tm_o);
     }
   }
+  if (threadIdx.x == 64) KD_EV(25);
   if (warp >= 2 && p.splits > 1 && !named_bar_red_or(1, GROUP, !ok || *cx.abort_flag))
     merge_splits(cx, p, cid, rank, PAGED);
+  if (threadIdx.x == 64) KD_EV(27);
 
   // ------------------------------------------------------- teardown
   __syncwarp();          // the roles leave lanes behind (single-lane issuers, lane 64's waits)
   __syncthreads();
   cluster_sync();
+  if (threadIdx.x == 0) KD_EV(2);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+    if (lane == 0) KD_EV(3);
   }
 }
 
@@ -1514,6 +1622,25 @@ int default_splits(int B, int n, int H, int64_t cap) {
 }  // namespace kd
 
 using namespace kd;
+
+#ifdef KD_TRACE
+// Trace build only: copy out / clear the per-CTA trace of the last launches.
+extern "C" int kd_trace_read(unsigned long long* host, size_t bytes) {
+  if (bytes > sizeof(tc::g_trace)) bytes = sizeof(tc::g_trace);
+  return cuda_status(cudaMemcpyFromSymbol(host, tc::g_trace, bytes), "cudaMemcpyFromSymbol(trace)");
+}
+extern "C" int kd_trace_clear(cudaStream_t stream) {
+  void* ptr = nullptr;
+  int st = cuda_status(cudaGetSymbolAddress(&ptr, tc::g_trace), "cudaGetSymbolAddress(trace)");
+  if (st) return st;
+  return cuda_status(cudaMemsetAsync(ptr, 0, sizeof(tc::g_trace), stream), "cudaMemsetAsync(trace)");
+}
+extern "C" int kd_trace_dims(int* ctas, int* slots) {
+  *ctas = tc::TRACE_CTAS;
+  *slots = tc::TRACE_SLOTS;
+  return KD_OK;
+}
+#endif
 
 extern "C" size_t kd_verify_workspace_bytes(int B, int n, int H, int64_t cap, int kv_splits) {
   if (!shapes_ok(B, n) || H < 1 || H > KD_MAX_HEADS || cap < 1 || kv_splits < 0 || kv_splits > 64) return 0;

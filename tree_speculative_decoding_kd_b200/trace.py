@@ -1,0 +1,188 @@
+"""Timeline and wait counters of attention launches, from the trace build.
+
+    python -m tree_speculative_decoding_kd_b200.build --trace
+    python -m tree_speculative_decoding_kd_b200.trace --configs tiny,kimi_single,batched
+
+libkdverify_trace.so is the library with the attention kernel compiled with
+-DKD_TRACE: per CTA it records the global timer at fixed points of each role and
+cycle counters of the main waits.  For each configuration the call is captured in a
+CUDA graph and replayed (warm, and after an L2 flush); this prints, per mode, the
+median replay's event time, the kernel's own span, the timeline of the cluster that
+finished last, and the per-tile / per-unit wait cycles of the roles.  A replay of a
+graph holding one tiny memset gives the event-timing floor (graph launch overhead).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+
+import numpy as np
+import torch
+
+from . import harness as HN
+from . import kd
+from . import workload as W
+
+# timeline slots (global timer, ns) and counter slots (SM cycles), as the kernel fills them
+EVENTS = {0: "entry", 1: "setup done (barriers, TMEM, cluster sync)", 2: "teardown sync", 3: "exit (TMEM freed)",
+          4: "QK producer: first unit claimed", 5: "QK producer: first Q loads issued",
+          6: "QK producer: first unit published", 7: "QK producer: last K load issued",
+          8: "QK MMA: first Q in TMEM", 9: "QK MMA: first K chunk landed", 10: "QK MMA: first S committed",
+          11: "QK MMA: last S committed", 12: "softmax: first Q copied to TMEM", 13: "softmax: first S loaded",
+          14: "softmax: first tile's P emitted", 15: "softmax: last S ready", 16: "softmax: last tile masked",
+          17: "softmax: last tile's P emitted", 18: "softmax: last row statistics sent",
+          19: "PV producer: first V issued", 20: "PV MMA: first P landed", 21: "PV MMA: last O complete (commit)",
+          22: "epilogue: last O and statistics ready", 23: "epilogue: last unit's first O chunk read",
+          24: "epilogue: last unit stored", 25: "merge: start", 26: "merge: first ticket complete",
+          27: "merge: end"}
+QK_COUNTERS = {32: ("QK MMA waits for S to be free", "tile"), 33: ("QK MMA waits for K stages", "tile"),
+               34: ("QK MMA issue (fence, MMAs, commits)", "tile"),
+               36: ("QK MMA unit start (unit decode to Q ready)", "unit"),
+               37: ("QK MMA waits for Q in TMEM", "unit"), 40: ("softmax waits for S", "tile"),
+               41: ("softmax emits P (two halves)", "tile"), 42: ("softmax tile total", "tile")}
+PV_COUNTERS = {44: ("PV MMA waits for P", "P half-tile"), 45: ("PV MMA waits for V", "P half-tile")}
+
+
+def _load():
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkdverify_trace.so")
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m tree_speculative_decoding_kd_b200.build --trace`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in kd._SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    lib.kd_trace_read.argtypes = [ctypes.c_void_p, ctypes.c_size_t]
+    lib.kd_trace_clear.argtypes = [ctypes.c_void_p]
+    lib.kd_trace_dims.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    c, s = ctypes.c_int(), ctypes.c_int()
+    lib.kd_trace_dims(ctypes.byref(c), ctypes.byref(s))
+    kd.lib = lib                       # every kd.* call below runs the trace build
+    return lib, c.value, s.value
+
+
+def _replays(call, flush, flushed, lib, dims, reps=7):
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    runs = []
+    for _ in range(reps):
+        s = torch.cuda.current_stream()
+        lib.kd_trace_clear(s.cuda_stream)
+        torch.cuda.synchronize()
+        if flushed:
+            flush()                    # keeps the GPU busy while the replay is enqueued
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        tr = np.zeros(dims, np.uint64)
+        lib.kd_trace_read(tr.ctypes.data, tr.nbytes)
+        runs.append((e0.elapsed_time(e1) * 1e3, tr.astype(np.int64)))
+    del g
+    runs.sort(key=lambda r: r[0])
+    return runs[len(runs) // 2]
+
+
+def _summary(t_ev, tr):
+    used = np.nonzero(tr[:, 0])[0]
+    tr = tr[: int(used.max()) + 1]
+    t0 = tr[:, 0][tr[:, 0] > 0].min()
+    res = {"event_us": round(t_ev, 2), "ctas": int(len(tr)),
+           "kernel_us (first entry to last exit)": round((tr[:, 3].max() - t0) / 1e3, 2)}
+    last = int(np.argmax(tr[1::2, 3])) if len(tr) > 1 else 0
+    tl = []
+    for cta in (2 * last, 2 * last + 1):
+        for i, name in EVENTS.items():
+            if cta < len(tr) and tr[cta, i] > 0 and (i > 3 or cta % 2 == 0):
+                tl.append((round((tr[cta, i] - t0) / 1e3, 2), ("QK CTA " if cta % 2 == 0 else "PV CTA ") + name
+                           if i in (0, 1, 2, 3, 25, 26, 27) else name))
+    res["timeline_us (cluster that finished last)"] = dict((n, t) for t, n in sorted(tl))
+    qk, pv = tr[0::2], tr[1::2]
+    tiles, units, halves = qk[:, 35].sum(), qk[:, 38].sum(), pv[:, 46].sum()
+    cyc = {}
+    for i, (name, per) in QK_COUNTERS.items():
+        den = tiles if per == "tile" else units
+        cyc[f"{name} (per {per})"] = round(float(qk[:, i].sum()) / max(den, 1), 1)
+    for i, (name, per) in PV_COUNTERS.items():
+        cyc[f"{name} (per {per})"] = round(float(pv[:, i].sum()) / max(halves, 1), 1)
+    res["tiles"], res["units"] = int(tiles), int(units)
+    res["cycles"] = cyc
+    return res
+
+
+def trace_config(name, lib, dims, flush, splits=0):
+    wl = W.make_workload(name)
+    cfg, st = wl.cfg, wl.step
+    qa, qr = kd.bf16_from_bits(st.q_abs), kd.bf16_from_bits(st.q_rope)
+    ck, kr = kd.bf16_from_bits(wl.c_kv), kd.bf16_from_bits(wl.k_rope)
+    lens = torch.from_numpy(wl.cache_lens.astype(np.int32)).cuda()
+    vis, _ = kd.kd_tree_build_mask(torch.from_numpy(st.parents).cuda())
+    ws = kd.new_workspace(cfg.B, cfg.n, cfg.H, cfg.cap, splits)
+    out = torch.empty(cfg.B, cfg.n, cfg.H, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(cfg.B, cfg.n, cfg.H, dtype=torch.float32, device="cuda")
+
+    def call():
+        kd.kd_tree_verify_attn(qa, qr, ck, kr, lens, vis, None, cfg.scale, out, lse, ws, kv_splits=splits)
+
+    res = []
+    for flushed in (False, True):
+        t, tr = _replays(call, flush, flushed, lib, dims)
+        res.append({"config": name, "splits": splits or "auto", "mode": "flushed" if flushed else "warm",
+                    **_summary(t, tr)})
+    bits = kd.kd_read_device_error(ws)
+    if bits:
+        raise RuntimeError(f"{name}: device error bits {bits:#x}")
+    return res
+
+
+def graph_floor(flush):
+    """Event time of a replayed graph that holds one 4-byte memset."""
+    z = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = []
+    for flushed in (False, True):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            z.zero_()
+        ts = []
+        for _ in range(7):
+            torch.cuda.synchronize()
+            if flushed:
+                flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        out.append({"graph_with_one_memset": "flushed" if flushed else "warm",
+                    "event_us": round(float(np.median(ts)), 2)})
+        del g
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--configs", default="tiny,kimi_single,batched")
+    ap.add_argument("--json", default=None, help="also write the results to this file")
+    args = ap.parse_args()
+    lib, ctas, slots = _load()
+    flush = HN.L2Flush("cuda")
+    res = graph_floor(flush)
+    for name in args.configs.split(","):
+        res += trace_config(name, lib, (ctas, slots), flush)
+    for r in res:
+        print(json.dumps(r))
+    if args.json:
+        with open(args.json, "w") as f:
+            json.dump(res, f, indent=1)
+
+
+if __name__ == "__main__":
+    main()
