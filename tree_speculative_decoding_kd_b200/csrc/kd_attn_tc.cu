@@ -535,10 +535,19 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, const Params& p, const int
   KD_CTR(c_us);
   KD_CTR(c_qt);
   KD_CTR(c_nu);
+  KD_CTR(c_f1);
+  KD_CTR(c_sc);
+  KD_CTR(c_tot);
+  KD_T0(tall);
+  KD_CTR(c_sw);
+  KD_CTR(c_tile);
+  KD_CTR(c_loop);
   for (int k = 0; ok; ++k) {
+    KD_T0(tw);
     if (!(ok = wait_bar(cx, cx.bar(SCHED_FULL + k % NS), (k / NS) & 1, true))) break;
     const int64_t r = slots[k % NS];
     sched_release(cx, k % NS, false);
+    if (k > 0) KD_ADD(c_sw, tw);
     if (r < 0) break;
     KD_T0(tu);
     const Unit u = unit_at(p, order, r);
@@ -550,15 +559,18 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, const Params& p, const int
     KD_INC(c_nu);
     if (uq == 0) KD_EV(8);
     tc_fence_after();
+    KD_T0(tl);
     for (int t = 0; t < u.ntiles && ok; ++t, ++ts) {
       KD_T0(te);
       if (!(ok = wait_bar(cx, cx.bar(S_EMPTY), (ts & 1u) ^ 1u))) break;
       KD_ADD(c_se, te);
       KD_INC(c_nt);
+      KD_T0(tf);
       tc_fence_after();
       const uint32_t d = tmem + TS;
       for (int c = 0; c < NCHUNK; ++c, ++it) {
         const uint32_t st = it % NK;
+        if (c == 0) KD_ADD(c_f1, tf);
         KD_T0(tk);
         if (!(ok = wait_bar(cx, cx.bar(K_FULL + st), (it / NK) & 1u))) break;
         KD_ADD(c_kf, tk);
@@ -578,10 +590,14 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, const Params& p, const int
         tc_commit(cx.bar(K_EMPTY + st));
         KD_ADD(c_is, ti);
       }
+      KD_T0(tc);
       if (ok) tc_commit(cx.bar(S_FULL));
+      KD_ADD(c_sc, tc);
+      KD_ADD(c_tile, te);
       if (ts == 0) KD_EV(10);
       KD_EV(11);
     }
+    KD_ADD(c_loop, tl);
     if (ok) tc_commit(cx.bar(Q_FREE));
     ++uq;
   }
@@ -592,6 +608,13 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, const Params& p, const int
   KD_FLUSH(36, c_us);
   KD_FLUSH(37, c_qt);
   KD_FLUSH(38, c_nu);
+  KD_FLUSH(47, c_f1);
+  KD_FLUSH(48, c_sc);
+  KD_FLUSH(50, c_sw);
+  KD_FLUSH(51, c_tile);
+  KD_FLUSH(52, c_loop);
+  KD_ADD(c_tot, tall);
+  KD_FLUSH(49, c_tot);
   tc_commit(cx.bar(DRAIN));
   wait_bar(cx, cx.bar(DRAIN), 0, false, true);
 }

@@ -41,7 +41,13 @@ QK_COUNTERS = {32: ("QK MMA waits for S to be free", "tile"), 33: ("QK MMA waits
                34: ("QK MMA issue (fence, MMAs, commits)", "tile"),
                36: ("QK MMA unit start (unit decode to Q ready)", "unit"),
                37: ("QK MMA waits for Q in TMEM", "unit"), 40: ("softmax waits for S", "tile"),
-               41: ("softmax emits P (two halves)", "tile"), 42: ("softmax tile total", "tile")}
+               41: ("softmax emits P (two halves)", "tile"), 42: ("softmax tile total", "tile"),
+               47: ("QK MMA fence after S is free (to the first K wait)", "tile"),
+               48: ("QK MMA commit of S", "tile"), 49: ("QK MMA role total", "tile"),
+               50: ("QK MMA waits for the next unit's schedule slot", "unit"),
+               51: ("QK MMA whole tile (S wait to S commit)", "tile"), 52: ("QK MMA tile loops", "tile")}
+# The whole-tile counter minus its timed parts is the time the MMA thread spends blocked between
+# them, i.e. in the issue of MMAs the tensor pipe is not yet ready to accept.
 PV_COUNTERS = {44: ("PV MMA waits for P", "P half-tile"), 45: ("PV MMA waits for V", "P half-tile")}
 
 
