@@ -4,7 +4,8 @@
     python -m tree_speculative_decoding_kd_b200.build --trace   # + libkdverify_trace.so
 
 The trace build compiles the attention with -DKD_TRACE: the same kernel recording a
-per-CTA timeline and wait counters of each launch (read by trace.py).
+per-CTA timeline and wait counters of each launch (read by trace.py), plus the L2
+delivery probes of csrc/kd_probe.cu.
 """
 from __future__ import annotations
 
@@ -72,6 +73,7 @@ def build_trace(verbose: bool = False) -> str:
     build(verbose)
     objs = [os.path.join(OBJ, os.path.splitext(s)[0] + ".o") for s in SOURCES if s != "kd_attn_tc.cu"]
     objs.append(_compile("kd_attn_tc.cu", verbose, ["-DKD_TRACE"], "_trace"))
+    objs.append(_compile("kd_probe.cu", verbose, ["-DKD_TRACE"], "_trace"))     # delivery probes
     tmp = TRACE_LIB + ".tmp"
     r = subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static"], capture_output=True,
                        text=True)

@@ -1,0 +1,222 @@
+// Delivery probes of the trace build (libkdverify_trace.so only; the product library
+// does not contain this file).
+//
+// How many bytes per SM cycle TMA tile loads deliver from an L2-resident window when a
+// ring of `depth` boxes is kept in flight, issued and waited on the way the attention's
+// K ring is (one thread issues; a stage is reused once its previous load landed; waits
+// poll the barrier and read the global timer once per 64 polls):
+//   - kd_probe_l2_boxes, pair = 0: one CTA per SM, each loading whole boxes;
+//   - pair = 1: 2-CTA clusters whose CTAs each load half of every box into their own
+//     shared memory, both halves completing on the even CTA's barrier (the load form a
+//     pair-MMA design would use for its B operand: cta_group::2, no multicast); the
+//     even CTA hands each stage back to the odd one with a remote arrive.
+// Every wait is bounded (2 s); one that gives up sets *err and the CTA drains and exits.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "kd_common.cuh"
+#include "kd_ptx.cuh"
+
+namespace kd {
+namespace probe {
+
+using namespace ptx;
+
+constexpr int MAX_DEPTH = 24;
+constexpr uint64_t LIMIT_NS = 2000000000ull;
+
+__device__ __forceinline__ bool poll(uint32_t bar, uint32_t parity, bool cluster_scope) {
+  uint64_t t0 = 0;
+  for (uint32_t spin = 0;; ++spin) {
+    if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if ((spin & 63u) == 63u) {
+      const uint64_t t = globaltimer();
+      if (t0 == 0) t0 = t;
+      else if (t - t0 > LIMIT_NS) return false;
+    }
+  }
+}
+
+// The pair form of the tiled load: the destination is this CTA's shared memory, the
+// barrier may be the peer's (cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* map, int32_t x, int32_t y,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+
+// Shared memory: FULL barriers at base, EMPTY barriers at base + 256, stages from
+// base + 1024 (1024-byte aligned, `stage_bytes` apart).
+// With `issuers` warps, warp w's lane 0 runs its own ring of depth / issuers stages
+// (its own barriers, stages and rows), so the CTA keeps `depth` boxes in flight either way.
+__global__ void __launch_bounds__(64, 1)
+l2_box_kernel(const __grid_constant__ CUtensorMap tm, int box_rows, int depth, int iters, int window_rows,
+              unsigned long long* cycles, int* err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t stage_bytes = (uint32_t)box_rows * 128u;
+  const int issuers = blockDim.x / 32, w = threadIdx.x >> 5;
+  const int all_stages = depth;
+  depth /= issuers;
+  const uint32_t base0 = (raw + 1023u) & ~1023u;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < all_stages; ++s) mbar_init(base0 + 8u * s, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // warp w: barriers from base0 + 8 (w depth), stages from base0 + 1024 + w depth stage_bytes
+  const uint32_t base = base0 + 8u * w * depth;
+  const uint32_t stages = base0 + 1024u + (uint32_t)(w * depth) * stage_bytes;
+  if ((threadIdx.x & 31) == 0) {
+    // no division in the loop: the row advances by one box and wraps; stage s and the
+    // parity of its next completion are counters
+    int y = (int)(((long long)(blockIdx.x * issuers + w) * 7919 * box_rows) % window_rows);
+    bool ok = true;
+    uint32_t par = 0;                        // parity of stage s's next completion, bit per stage
+    const long long t0 = clock64();
+    int i = 0, s = 0;
+    for (; i < iters && ok; ++i) {
+      if (i >= depth) {
+        if (!(ok = poll(base + 8u * s, (par >> s) & 1u, false))) break;
+        par ^= 1u << s;
+      }
+      mbar_arrive_expect_tx(base + 8u * s, stage_bytes);
+      tma_load_2d(stages + s * stage_bytes, &tm, 0, y, base + 8u * s);
+      y += box_rows;
+      if (y >= window_rows) y -= window_rows;
+      if (++s == depth) s = 0;
+    }
+    for (int j = 0; j < depth && j < i; ++j) {     // the last loads, in issue order from stage s
+      if (!poll(base + 8u * s, (par >> s) & 1u, false)) ok = false;
+      par ^= 1u << s;
+      if (++s == depth) s = 0;
+    }
+    atomicMax(cycles + blockIdx.x, (unsigned long long)(clock64() - t0));
+    if (!ok) atomicOr(err, 1);
+  }
+  __syncthreads();
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(32, 1)
+l2_pair_kernel(const __grid_constant__ CUtensorMap tm, int box_rows, int depth, int iters, int window_rows,
+               unsigned long long* cycles, int* err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t half_rows = (uint32_t)box_rows / 2;
+  const uint32_t stage_bytes = half_rows * 128u;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < depth; ++s) {
+      mbar_init(base + 8u * s, 1);          // FULL (used in the even CTA)
+      mbar_init(base + 256u + 8u * s, 1);   // EMPTY (used in the odd CTA)
+    }
+    fence_mbar_init();
+  }
+  cluster_sync();
+  const uint32_t full_even = map_to_rank(base, 0);        // FULL barriers of the even CTA
+  const uint32_t empty_odd = map_to_rank(base + 256u, 1);   // EMPTY barriers of the odd CTA
+  if (threadIdx.x == 0) {
+    int y = (int)(((long long)(blockIdx.x / 2) * 7919 * box_rows) % window_rows);
+    bool ok = true;
+    uint32_t par = 0;
+    const long long t0 = clock64();
+    int i = 0, s = 0;
+    for (; i < iters && ok; ++i) {
+      if (rank == 0) {
+        if (i >= depth) {
+          if (!(ok = poll(base + 8u * s, (par >> s) & 1u, true))) break;
+          mbar_arrive_remote(empty_odd + 8u * s);                 // the odd CTA may reuse stage s
+        }
+        mbar_arrive_expect_tx(base + 8u * s, 2u * stage_bytes);
+      } else if (i >= depth && !(ok = poll(base + 256u + 8u * s, (par >> s) & 1u, true))) {
+        break;
+      }
+      if (i >= depth) par ^= 1u << s;
+      tma_load_2d_pair(base + 1024u + s * stage_bytes, &tm, 0, y + (int)(rank * half_rows), full_even + 8u * s);
+      y += box_rows;
+      if (y >= window_rows) y -= window_rows;
+      if (++s == depth) s = 0;
+    }
+    // the even CTA waits for the last loads and releases their stages; the odd CTA
+    // waits for those releases, so neither leaves with a load in flight
+    for (int j = 0; j < depth && j < i; ++j) {
+      if (rank == 0) {
+        if (!poll(base + 8u * s, (par >> s) & 1u, true)) ok = false;
+        mbar_arrive_remote(empty_odd + 8u * s);
+      } else if (!poll(base + 256u + 8u * s, (par >> s) & 1u, true)) {
+        ok = false;
+      }
+      par ^= 1u << s;
+      if (++s == depth) s = 0;
+    }
+    cycles[blockIdx.x] = (unsigned long long)(clock64() - t0);
+    if (!ok) atomicOr(err, 1);
+  }
+  __syncwarp();
+  cluster_sync();
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+}  // namespace probe
+}  // namespace kd
+
+// buf: bf16 [rows][512] on the device (rows a multiple of box_rows); box_rows 32..256 (even),
+// depth 1..24 boxes in flight, pair 0 or 1.  cycles: device uint64 [grid CTAs]; err: device
+// int32 (ORed).  Grid: 148 CTAs (74 clusters when pair).
+extern "C" int kd_probe_l2_boxes(const void* buf, int rows, int box_rows, int depth, int iters, int pair,
+                                 unsigned long long* cycles, int* err, cudaStream_t stream) {
+  // pair: 0 whole boxes, one issuing warp; 1 pair loads; 2 whole boxes, two issuing warps
+  const int issuers = pair == 2 ? 2 : 1;
+  if (pair == 2) pair = 0;
+  if (depth % issuers) return KD_EINVAL;
+  using namespace kd::probe;
+  if (!buf || !cycles || !err || box_rows < 32 || box_rows > 256 || (box_rows & 1) || depth < 1 ||
+      depth > MAX_DEPTH || iters < depth || rows < box_rows || rows % box_rows)
+    return KD_EINVAL;
+  const size_t smem = 1024 + 1024 + (size_t)depth * box_rows * 128 / (pair ? 2 : 1);
+  if (smem > 232448) return KD_ERANGE;
+  auto fn = encode_fn();
+  if (!fn) return KD_ELAUNCH;
+  CUtensorMap tm;
+  cuuint64_t dims[2] = {512, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {1024};
+  cuuint32_t box[2] = {64, (cuuint32_t)(pair ? box_rows / 2 : box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(buf), dims, strides, box, es,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return KD_ELAUNCH;
+  int st;
+  if (pair) {
+    if ((st = kd::cuda_status(cudaFuncSetAttribute(l2_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)smem), "cudaFuncSetAttribute(probe)")))
+      return st;
+    l2_pair_kernel<<<148, 32, smem, stream>>>(tm, box_rows, depth, iters, rows, cycles, err);
+  } else {
+    if ((st = kd::cuda_status(cudaFuncSetAttribute(l2_box_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)smem), "cudaFuncSetAttribute(probe)")))
+      return st;
+    l2_box_kernel<<<148, 32 * issuers, smem, stream>>>(tm, box_rows, depth, iters / issuers, rows, cycles, err);
+  }
+  return kd::launch_status("l2 probe");
+}

@@ -10,6 +10,13 @@ CUDA graph and replayed (warm, and after an L2 flush); this prints, per mode, th
 median replay's event time, the kernel's own span, the timeline of the cluster that
 finished last, and the per-tile / per-unit wait cycles of the roles.  A replay of a
 graph holding one tiny memset gives the event-timing floor (graph launch overhead).
+
+    python -m tree_speculative_decoding_kd_b200.trace --probes
+
+runs the delivery probes of the same library instead: bytes per SM cycle that TMA tile
+loads deliver from an L2-resident window with a given number of boxes in flight, for
+whole boxes per CTA and for the pair form (two CTAs each loading half of every box,
+completing on the even CTA's barrier).
 """
 from __future__ import annotations
 
@@ -63,6 +70,8 @@ def _load():
     lib.kd_trace_read.argtypes = [ctypes.c_void_p, ctypes.c_size_t]
     lib.kd_trace_clear.argtypes = [ctypes.c_void_p]
     lib.kd_trace_dims.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    lib.kd_probe_l2_boxes.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
     c, s = ctypes.c_int(), ctypes.c_int()
     lib.kd_trace_dims(ctypes.byref(c), ctypes.byref(s))
     kd.lib = lib                       # every kd.* call below runs the trace build
@@ -173,16 +182,53 @@ def graph_floor(flush):
     return out
 
 
+def probes(lib, iters=3000):
+    """Delivery of TMA tile loads from an 8 MB L2-resident window, per SM cycle."""
+    rows = 8192
+    buf = torch.randn(rows, 512, device="cuda").to(torch.bfloat16)
+    cycles = torch.zeros(148, dtype=torch.int64, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = []
+    # pair: 0 whole boxes (one issuing warp), 1 pair loads, 2 whole boxes from two issuing warps
+    cases = [(0, 64, 16), (0, 128, 8), (0, 256, 4), (0, 256, 6),
+             (2, 64, 16), (2, 128, 8), (2, 256, 4), (2, 256, 6),
+             (1, 64, 24), (1, 128, 16), (1, 256, 8)]
+    names = {0: "whole boxes, one issuing thread", 1: "pair: half boxes, even CTA's barrier",
+             2: "whole boxes, two issuing warps"}
+    for pair, box_rows, depth in cases:
+        for _ in range(2):                     # the first run brings the window into L2
+            cycles.zero_()
+            rc = lib.kd_probe_l2_boxes(buf.data_ptr(), rows, box_rows, depth, iters, pair, cycles.data_ptr(),
+                                       err.data_ptr(), torch.cuda.current_stream().cuda_stream)
+            if rc != 0:
+                raise RuntimeError(f"probe rc {rc}")
+            torch.cuda.synchronize()
+        if int(err.item()) != 0:
+            raise RuntimeError("a probe wait gave up")
+        half = 2 if pair == 1 else 1
+        per_cta_bytes = iters * box_rows * 128 // half
+        bpc = per_cta_bytes / cycles.cpu().numpy().astype(np.float64)
+        out.append({"probe": names[pair], "box_rows": box_rows, "bytes_per_load": box_rows * 128 // half,
+                    "in_flight_KB_per_SM": depth * box_rows * 128 // half // 1024,
+                    "B_per_SM_cycle_median": round(float(np.median(bpc)), 1),
+                    "B_per_SM_cycle_min": round(float(bpc.min()), 1)})
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--configs", default="tiny,kimi_single,batched")
+    ap.add_argument("--probes", action="store_true", help="run the L2 delivery probes instead")
     ap.add_argument("--json", default=None, help="also write the results to this file")
     args = ap.parse_args()
     lib, ctas, slots = _load()
-    flush = HN.L2Flush("cuda")
-    res = graph_floor(flush)
-    for name in args.configs.split(","):
-        res += trace_config(name, lib, (ctas, slots), flush)
+    if args.probes:
+        res = probes(lib)
+    else:
+        flush = HN.L2Flush("cuda")
+        res = graph_floor(flush)
+        for name in args.configs.split(","):
+            res += trace_config(name, lib, (ctas, slots), flush)
     for r in res:
         print(json.dumps(r))
     if args.json:
