@@ -68,9 +68,11 @@ def build(verbose: bool = False, force: bool = False) -> str:
     return LIB
 
 
-def build_trace(verbose: bool = False) -> str:
+def build_trace(verbose: bool = False, force: bool = False) -> str:
     """libkdverify_trace.so: the library with the attention compiled with -DKD_TRACE."""
-    build(verbose)
+    lib = build(verbose)
+    if not force and os.path.exists(TRACE_LIB) and os.path.getmtime(TRACE_LIB) >= os.path.getmtime(lib):
+        return TRACE_LIB
     objs = [os.path.join(OBJ, os.path.splitext(s)[0] + ".o") for s in SOURCES if s != "kd_attn_tc.cu"]
     objs.append(_compile("kd_attn_tc.cu", verbose, ["-DKD_TRACE"], "_trace"))
     objs.append(_compile("kd_probe.cu", verbose, ["-DKD_TRACE"], "_trace"))     # delivery probes
@@ -86,4 +88,4 @@ def build_trace(verbose: bool = False) -> str:
 if __name__ == "__main__":
     print(build(verbose="-v" in sys.argv, force=True))
     if "--trace" in sys.argv:
-        print(build_trace(verbose="-v" in sys.argv))
+        print(build_trace(verbose="-v" in sys.argv, force=True))
