@@ -1114,7 +1114,7 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
     // all issued, which O being complete implies, so this peek at the next schedule
     // slot cannot wait on anything the epilogue still has to do.  With no next unit
     // the P slots and the V ring are idle for good, and this unit's stores stage
-    // through them (EPI_RING slots per warp, 64 columns per round) instead of
+    // through them (EPI_RING slots per warp, 64 columns per pass) instead of
     // through the warp's single 2 KB slot.
     const int kn = k + 1;
     if (!(ok = wait_group(cx, cx.bar(SCHED_FULL + kn % NS), (kn / NS) & 1, true))) break;
@@ -1137,8 +1137,8 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
     // Rolled loops over small TMEM reads: this code runs once per unit, so its size
     // (fetched cold every time) matters more than the exposed TMEM read latency.
     if (last) {
-      // 64 columns per round: two bf16 boxes or four fp32 boxes, one fence and one
-      // commit group per round; slots (round * boxes + j) % EPI_RING
+      // 64 columns per pass: two bf16 boxes or four fp32 boxes, one fence and one
+      // commit group per pass; slots (pass * boxes + j) % EPI_RING
 #pragma unroll 1
       for (int c = 0; c < 256 / 64; ++c) {
         uint32_t v[64];
@@ -1149,7 +1149,7 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
           tc_fence_before();
           mbar_arrive(cx.bar(O_FREE));
         }
-        // fp32 round 3 reuses round 0's slots: its boxes must be read out first
+        // fp32 pass 3 reuses pass 0's slots: its boxes must be read out first
         if (lane == 0 && p.splits > 1 && c == 3) bulk_wait_group_read<2>();
         __syncwarp();
         if (p.splits == 1) {
