@@ -182,6 +182,7 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(QSTAGES * KCHUNK == NQT * CHUNK && QSTAGES <= NK, "Q latent through the ring");
 
 constexpr uint32_t IDESC_QK = idesc_bf16(BM, BQ, 0, 0);    // Q, K both K-major
+constexpr uint32_t IDESC_QK_HALF = idesc_bf16(BM, BN, 0, 0); // a tile's first 128 keys only
 constexpr uint32_t IDESC_PV = idesc_bf16(BM, 256, 0, 1);   // P K-major, V MN-major
 constexpr float RESCALE_THRESHOLD = 8.0f;                  // log2 units: P <= 2^8
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;          // 2 s per wait
@@ -568,6 +569,9 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, const Params& p, const int
       KD_T0(tf);
       tc_fence_after();
       const uint32_t d = tmem + TS;
+      // a tile whose second half lies past the last key needs only its first 128 keys'
+      // scores (the softmax masks the other columns, whatever they hold)
+      const uint32_t idesc = u.kbeg + (int64_t)t * BQ + BN < u.nkeys ? IDESC_QK : IDESC_QK_HALF;
       for (int c = 0; c < NCHUNK; ++c, ++it) {
         const uint32_t st = it % NK;
         if (c == 0) KD_ADD(c_f1, tf);
@@ -581,11 +585,11 @@ __device__ __forceinline__ void qk_mma(const Ctx& cx, const Params& p, const int
         if (c < NQT) {
 #pragma unroll
           for (int kk = 0; kk < KC / 16; ++kk)
-            mma_bf16_ts(d, tmem + TQ + c * 32 + kk * 8, desc_k(b0 + kk * 32), IDESC_QK, (c | kk) != 0);
+            mma_bf16_ts(d, tmem + TQ + c * 32 + kk * 8, desc_k(b0 + kk * 32), idesc, (c | kk) != 0);
         } else {
 #pragma unroll
           for (int kk = 0; kk < KC / 16; ++kk)
-            mma_bf16_ss(d, desc_k(base + Q_OFF + kk * 32), desc_k(b0 + kk * 32), IDESC_QK, 1u);
+            mma_bf16_ss(d, desc_k(base + Q_OFF + kk * 32), desc_k(b0 + kk * 32), idesc, 1u);
         }
         tc_commit(cx.bar(K_EMPTY + st));
         KD_ADD(c_is, ti);
@@ -837,9 +841,14 @@ __device__ __forceinline__ bool qk_softmax(const Ctx& cx, const Params& p, const
             ok = wait_group(cx, cx.bar(Q_FREE), nq & 1u) &&
                  copy_q(cx, gbase, lane_addr, pos + QSTAGES + NCHUNK * (uint32_t)u.ntiles, g, r);
         }
-        ok = ok && emit_p(cx, gbase, x[1], pc + 1, p.scale_log2, mb, 1.f, false, r, g, peer_p, peer_ctrl,
-                          l_part);
-        pc += 2;
+        // the second half may lie wholly past the last key: then it is not sent
+        if (u.kbeg + (int64_t)t * BQ + BN < u.nkeys) {
+          ok = ok && emit_p(cx, gbase, x[1], pc + 1, p.scale_log2, mb, 1.f, false, r, g, peer_p, peer_ctrl,
+                            l_part);
+          pc += 2;
+        } else {
+          pc += 1;
+        }
         KD_ADD(c_em, tem);
         KD_ADD(c_tt, tsf);
         if (threadIdx.x == 64) {
@@ -955,7 +964,10 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int
     const Unit u = unit_at(p, order, r);
     // the epilogue must have read the previous unit's O before it is overwritten
     if (vu > 0 && !(ok = wait_warp(cx, cx.bar(O_FREE), (vu - 1) & 1u))) break;
-    for (int t = 0; t < 2 * u.ntiles && ok; ++t, ++pc) {      // P tiles of 128 keys
+    for (int t = 0; t < 2 * u.ntiles && ok; ++t) {            // P tiles of 128 keys
+      // a P tile wholly past the request's last key (the second half of a tile) is
+      // neither sent by the QK CTA nor multiplied here; pc counts the tiles exchanged
+      if (u.kbeg + (int64_t)t * BN >= u.nkeys) continue;
       const uint32_t sb = pc & 1;
       if (lane == 0) mbar_arrive_expect_tx(cx.bar(P_FULL + sb), SLOT_COPY);
       KD_T0(tp);
@@ -1014,6 +1026,7 @@ __device__ __forceinline__ void pv_mma(const Ctx& cx, const Params& p, const int
       }
       if (ok && lane == 0) tc_commit_mc(cx.bar(P_FREE + sb), (uint16_t)(1u << cx.peer));
       __syncwarp();
+      ++pc;
     }
     if (!ok) break;
     if (lane == 0) {
