@@ -1092,6 +1092,9 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
   volatile int64_t* slots = sched_slots(gbase);
   bool ok = true;
   uint32_t nev = 0, vu = 0;
+  KD_CTR(c_es);
+  KD_CTR(c_ew);
+  KD_CTR(c_eu);
   for (int k = 0; ok; ++k) {
     if (!(ok = wait_group(cx, cx.bar(SCHED_FULL + k % NS), (k / NS) & 1, true))) break;
     const int64_t rk = slots[k % NS];
@@ -1147,6 +1150,7 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
     const bool store = pages_ok && R0w < rows_req;
     const int z = p.splits == 1 ? u.b : u.sp * p.B + u.b;
     const uint32_t stg = last ? cx.base + P_OFF + (warp - 2) * (EPI_RING * 2048) : cx.base + EPI_OFF + (warp - 2) * 2048;
+    KD_T0(tes);
     // Rolled loops over small TMEM reads: this code runs once per unit, so its size
     // (fetched cold every time) matters more than the exposed TMEM read latency.
     if (last) {
@@ -1233,6 +1237,8 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
       else p.part_lse[(int64_t)u.sp * p.B * rows_req + grow] = lse_v;
     }
     if (p.splits > 1) {
+      KD_ADD(c_es, tes);
+      KD_T0(tew);
       // the partial is in global memory once every warp's boxes are written: publish
       // it on the tile's ticket
       if (lane == 0) {
@@ -1244,12 +1250,19 @@ __device__ __forceinline__ bool pv_epilogue(const Ctx& cx, const Params& p, cons
         __threadfence();
         atom_add_release_gpu(p.tickets + 2 * ((int64_t)u.b * p.mtiles + u.mt), 1);
       }
+      KD_ADD(c_ew, tew);
+      KD_INC(c_eu);
     }
     if (threadIdx.x == 64) KD_EV(24);
     ++vu;
   }
   if (lane == 0) bulk_wait_group0();            // every box stored before the CTA leaves
   __syncwarp();
+  if (threadIdx.x == 64) {
+    KD_FLUSH(58, c_es);
+    KD_FLUSH(59, c_ew);
+    KD_FLUSH(60, c_eu);
+  }
   return ok;
 }
 
@@ -1290,6 +1303,10 @@ __device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, int
   const uint32_t mbuf = cx.base + (rank == 0 ? STG_OFF : P_OFF);
   const int batch_rows = MBUF_ROWS / S;                      // S <= 64 < MBUF_ROWS
   uint32_t mph = 0;
+  KD_CTR(c_mt);
+  KD_CTR(c_ml);
+  KD_CTR(c_mc);
+  KD_CTR(c_mn);
   for (int row0 = a; row0 < e;) {
     const int b = row0 / rows_req;
     const int R0 = row0 - b * rows_req;
@@ -1310,6 +1327,7 @@ __device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, int
       const int busy = __popcll(busy_mask);
       int32_t* ticket = p.tickets + 2 * ((int64_t)b * p.mtiles + mt);
       // wait until every busy partition of the tile has stored its partial
+      KD_T0(tmt);
       bool ok = true;
       if (tid == 0) {
         uint64_t t0 = 0;
@@ -1323,6 +1341,8 @@ __device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, int
         }
       }
       if (named_bar_red_or(1, GROUP, !ok)) return;
+      KD_ADD(c_mt, tmt);
+      KD_INC(c_mn);
 #ifdef KD_TRACE
       if (threadIdx.x == 64 && g_trace[blockIdx.x][26] == 0) KD_EV(26);
 #endif
@@ -1354,9 +1374,12 @@ __device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, int
           if (s0) l0n = __ldcg(p.part_lse + (int64_t)lane * rows_all + (bs + rw + GROUP / 32));
           if (s1) l1n = __ldcg(p.part_lse + (int64_t)(lane + 32) * rows_all + (bs + rw + GROUP / 32));
         }
+        KD_T0(tml);
         const bool landed = wait_bar(cx, cx.bar(MERGE_FULL), mph & 1u, false, true);
         ++mph;
         if (named_bar_red_or(1, GROUP, !landed)) { abort_pair(cx); return; }
+        KD_ADD(c_ml, tml);
+        KD_T0(tmc);
         for (int r = rw; r < nb; r += GROUP / 32) {
           const int grow = bs + r;
           if (r == rw + GROUP / 32) {
@@ -1400,6 +1423,7 @@ __device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, int
           if (lane == 0) p.lse[grow] = sum > 0.f ? mx + __logf(sum) : -INFINITY;
         }
         named_bar_sync(1, GROUP);               // the buffer is read out before the next batch
+        KD_ADD(c_mc, tmc);
       }
       const int mine = (int)(row1 - row0);
       if (tid == 0 && atomicAdd(ticket + 1, mine) + mine == rows_in) {
@@ -1408,6 +1432,12 @@ __device__ __forceinline__ void merge_splits(const Ctx& cx, const Params& p, int
       }
     }
     row0 = row1;
+  }
+  if (threadIdx.x == 64) {
+    KD_FLUSH(53, c_mt);
+    KD_FLUSH(54, c_ml);
+    KD_FLUSH(55, c_mc);
+    KD_FLUSH(56, c_mn);
   }
 }
 

@@ -56,6 +56,12 @@ QK_COUNTERS = {32: ("QK MMA waits for S to be free", "tile"), 33: ("QK MMA waits
 # The whole-tile counter minus its timed parts is the time the MMA thread spends blocked between
 # them, i.e. in the issue of MMAs the tensor pipe is not yet ready to accept.
 PV_COUNTERS = {44: ("PV MMA waits for P", "P half-tile"), 45: ("PV MMA waits for V", "P half-tile")}
+# split-KV only: the epilogue's partial store (PV CTA, per unit) and the merge (both CTAs, per
+# M tile merged; slot 56 counts them)
+STORE_COUNTERS = {58: "epilogue: read O, stage and issue the partial's stores",
+                  59: "epilogue: wait for the partial's stores to complete, publish the ticket"}
+MERGE_COUNTERS = {53: "merge: wait for the tile's ticket", 54: "merge: wait for the partial rows to land",
+                  55: "merge: combine rows and store"}
 
 
 def _load():
@@ -127,6 +133,13 @@ def _summary(t_ev, tr):
         cyc[f"{name} (per {per})"] = round(float(qk[:, i].sum()) / max(den, 1), 1)
     for i, (name, per) in PV_COUNTERS.items():
         cyc[f"{name} (per {per})"] = round(float(pv[:, i].sum()) / max(halves, 1), 1)
+    su, mn = pv[:, 60].sum(), tr[:, 56].sum()
+    for i, name in STORE_COUNTERS.items():
+        if su > 0:
+            cyc[f"{name} (per unit)"] = round(float(pv[:, i].sum()) / su, 1)
+    for i, name in MERGE_COUNTERS.items():
+        if mn > 0:
+            cyc[f"{name} (per merged M tile, per CTA)"] = round(float(tr[:, i].sum()) / mn, 1)
     res["tiles"], res["units"] = int(tiles), int(units)
     res["cycles"] = cyc
     return res
