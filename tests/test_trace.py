@@ -59,3 +59,18 @@ def test_delivery_probe_runs(kd, traced):
         torch.cuda.synchronize()
         assert int(err.item()) == 0
         assert (cycles.cpu().numpy() > 0).all()
+
+
+def test_store_probe_covers_each_tile(kd, traced):
+    trace, lib, product, dims = traced
+    ctas = 4
+    cycles = torch.zeros(ctas, dtype=torch.int64, device="cuda")
+    for mode in (0, 1, 2):
+        buf = torch.ones(ctas, 128, 512, dtype=torch.float32, device="cuda")
+        rc = lib.kd_probe_store(buf.data_ptr(), ctas, mode, 2, cycles.data_ptr(),
+                                torch.cuda.current_stream().cuda_stream)
+        assert rc == 0
+        torch.cuda.synchronize()
+        assert (cycles.cpu().numpy() > 0).all()
+        assert int(torch.count_nonzero(buf)) == 0       # every element of every CTA's tile written
+    assert lib.kd_probe_store(buf.data_ptr(), 149, 0, 1, cycles.data_ptr(), None) != 0

@@ -11,6 +11,15 @@
 //     pair-MMA design would use for its B operand: cta_group::2, no multicast); the
 //     even CTA hands each stage back to the odd one with a remote arrive.
 // Every wait is bounded (2 s); one that gives up sets *err and the CTA drains and exits.
+//
+// kd_probe_store measures the other direction, in the attention epilogue's pattern: each CTA
+// writes a 128 x 512 fp32 tile (256 KB, one split partial) into its own plane, `reps` times
+// back to back, and waits once at the end for every store to complete:
+//   - mode 0: 8 warps, lane 0 of each issuing 2 KB TMA box stores (16 columns x 32 rows,
+//     64-byte swizzle) from its staging slot, as the epilogue does;
+//   - mode 1: the same in 4 KB boxes (32 columns x 32 rows, 128-byte swizzle);
+//   - mode 2: plain 16-byte stores from 256 threads, each warp instruction writing 512
+//     contiguous bytes of a row.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -164,6 +173,43 @@ l2_pair_kernel(const __grid_constant__ CUtensorMap tm, int box_rows, int depth, 
   cluster_sync();
 }
 
+// Shared memory: eight 4 KB staging slots (one per warp) from a 1024-byte aligned base; their
+// content is irrelevant and never rewritten, so a slot is reused without waiting for reads.
+__global__ void __launch_bounds__(256, 1)
+store_kernel(const __grid_constant__ CUtensorMap tm, float* buf, int mode, int reps, unsigned long long* cycles) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 8 * 4096 / 16; i += 256) st_shared_v4(base + i * 16, 0u, 0u, 0u, 0u);
+  fence_proxy_async_cta();
+  __syncthreads();
+  const long long t0 = clock64();
+  const int z = blockIdx.x;
+  const int row0 = (warp & 3) * 32, col0 = (warp >> 2) * 256;   // the warp's 32 rows x 256 columns
+  if (mode < 2) {
+    if (lane == 0) {
+      const int w = mode == 0 ? 16 : 32;                           // columns per box
+      for (int rep = 0; rep < reps; ++rep)
+        for (int c = 0; c < 256 / w; ++c) {
+          tma_store_3d(&tm, base + warp * 4096, col0 + c * w, row0, z);
+          bulk_commit_group();
+        }
+      bulk_wait_group0();
+    }
+    __syncwarp();
+  } else {
+    float* dst = buf + ((size_t)z * 128 + row0) * 512 + col0;
+    for (int rep = 0; rep < reps; ++rep)
+      for (int rr = 0; rr < 32; ++rr) {
+        st_global_v4(dst + rr * 512 + lane * 4, 0u, 0u, 0u, 0u);
+        st_global_v4(dst + rr * 512 + 128 + lane * 4, 0u, 0u, 0u, 0u);
+      }
+    __threadfence();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) cycles[blockIdx.x] = (unsigned long long)(clock64() - t0);
+}
+
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static std::once_flag once;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -219,4 +265,31 @@ extern "C" int kd_probe_l2_boxes(const void* buf, int rows, int box_rows, int de
     l2_box_kernel<<<148, 32 * issuers, smem, stream>>>(tm, box_rows, depth, iters / issuers, rows, cycles, err);
   }
   return kd::launch_status("l2 probe");
+}
+
+// buf: device fp32 [ctas][128][512]; ctas 1..148; mode 0..2; reps >= 1.  cycles: device uint64
+// [ctas] (SM cycles from the first store to the last completion, per CTA).
+extern "C" int kd_probe_store(void* buf, int ctas, int mode, int reps, unsigned long long* cycles,
+                              cudaStream_t stream) {
+  using namespace kd::probe;
+  if (!buf || !cycles || ctas < 1 || ctas > 148 || mode < 0 || mode > 2 || reps < 1) return KD_EINVAL;
+  auto fn = encode_fn();
+  if (!fn) return KD_ELAUNCH;
+  CUtensorMap tm;
+  const int w = mode == 1 ? 32 : 16;
+  cuuint64_t dims[3] = {512, 128, (cuuint64_t)ctas};
+  cuuint64_t strides[2] = {512 * 4, 128 * 512 * 4};
+  cuuint32_t box[3] = {(cuuint32_t)w, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, buf, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         mode == 1 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return KD_ELAUNCH;
+  const int smem = 8 * 4096 + 1024;
+  int st;
+  if ((st = kd::cuda_status(cudaFuncSetAttribute(store_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                            "cudaFuncSetAttribute(store probe)")))
+    return st;
+  store_kernel<<<ctas, 256, smem, stream>>>(tm, static_cast<float*>(buf), mode, reps, cycles);
+  return kd::launch_status("store probe");
 }

@@ -78,6 +78,8 @@ def _load():
     lib.kd_trace_dims.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     lib.kd_probe_l2_boxes.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    lib.kd_probe_store.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                   ctypes.c_void_p]
     c, s = ctypes.c_int(), ctypes.c_int()
     lib.kd_trace_dims(ctypes.byref(c), ctypes.byref(s))
     kd.lib = lib                       # every kd.* call below runs the trace build
@@ -225,6 +227,32 @@ def probes(lib, iters=3000):
                     "in_flight_KB_per_SM": depth * box_rows * 128 // half // 1024,
                     "B_per_SM_cycle_median": round(float(np.median(bpc)), 1),
                     "B_per_SM_cycle_min": round(float(bpc.min()), 1)})
+    out += store_probes(lib)
+    return out
+
+
+def store_probes(lib):
+    """Store rate of one 256 KB fp32 tile per CTA in the epilogue's pattern, per SM cycle."""
+    kinds = {0: "2 KB TMA box stores (16 fp32 columns x 32 rows), 8 issuing warps",
+             1: "4 KB TMA box stores (32 fp32 columns x 32 rows), 8 issuing warps",
+             2: "16-byte stores, 512 contiguous bytes per warp instruction"}
+    out = []
+    for ctas in (54, 148):
+        buf = torch.empty(ctas, 128, 512, dtype=torch.float32, device="cuda")
+        cycles = torch.zeros(ctas, dtype=torch.int64, device="cuda")
+        for mode in (0, 1, 2):
+            for reps in (1, 8):
+                for _ in range(2):
+                    rc = lib.kd_probe_store(buf.data_ptr(), ctas, mode, reps, cycles.data_ptr(),
+                                            torch.cuda.current_stream().cuda_stream)
+                    if rc != 0:
+                        raise RuntimeError(f"store probe rc {rc}")
+                    torch.cuda.synchronize()
+                bpc = reps * 128 * 512 * 4 / cycles.cpu().numpy().astype(np.float64)
+                out.append({"probe": "store: " + kinds[mode], "storing_ctas": ctas, "tiles_per_cta": reps,
+                            "cycles_median": int(np.median(cycles.cpu().numpy())),
+                            "B_per_SM_cycle_median": round(float(np.median(bpc)), 1)})
+        del buf
     return out
 
 
@@ -233,6 +261,8 @@ def main():
     ap.add_argument("--configs", default="tiny,kimi_single,batched")
     ap.add_argument("--probes", action="store_true", help="run the L2 delivery probes instead")
     ap.add_argument("--json", default=None, help="also write the results to this file")
+    ap.add_argument("--splits", default="0",
+                    help="comma-separated key-partition counts to trace each config at (0: automatic)")
     args = ap.parse_args()
     lib, ctas, slots = _load()
     if args.probes:
@@ -241,7 +271,8 @@ def main():
         flush = HN.L2Flush("cuda")
         res = graph_floor(flush)
         for name in args.configs.split(","):
-            res += trace_config(name, lib, (ctas, slots), flush)
+            for sp in args.splits.split(","):
+                res += trace_config(name, lib, (ctas, slots), flush, int(sp))
     for r in res:
         print(json.dumps(r))
     if args.json:
