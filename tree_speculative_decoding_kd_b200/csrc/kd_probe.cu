@@ -20,6 +20,14 @@
 //   - mode 1: the same in 4 KB boxes (32 columns x 32 rows, 128-byte swizzle);
 //   - mode 2: plain 16-byte stores from 256 threads, each warp instruction writing 512
 //     contiguous bytes of a row.
+//
+// kd_probe_mma measures the tensor pipe as its issuing threads see it: each CTA (one per SM)
+// issues `count` tcgen05.mma (kind::f16, bf16, M = 128, K = 16, N = 64 / 128 / 256) back to back
+// from one thread (or from two threads in two warps, each into its own accumulator) into TMEM,
+// A from shared memory or from TMEM, B from shared memory, and with
+// `wait_every` > 0 it polls an already-completed mbarrier after every `wait_every` MMAs (a
+// shared-memory read while MMAs are in flight, as a pipeline's per-stage wait is).  One commit
+// at the end; the cycles run from the first issue to that commit's arrival.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -210,6 +218,82 @@ store_kernel(const __grid_constant__ CUtensorMap tm, float* buf, int mode, int r
   if (threadIdx.x == 0) cycles[blockIdx.x] = (unsigned long long)(clock64() - t0);
 }
 
+// Shared memory from a 1024-byte aligned base: TMEM address at +0, barriers at +64 and +80
+// (done, one per issuer) and +72 (ready), A (128 rows x 64 bf16, 16 KB) at +1024, B (256 rows x 64 bf16, 32 KB) at
+// +17408; both zero, 128-byte swizzled K-major.  The dynamic size (> half an SM's) keeps one
+// CTA per SM, so the 512-column allocation never waits for another CTA.
+constexpr int MMA_SMEM = 120 * 1024;
+template <bool A_TMEM>
+__global__ void __launch_bounds__(128, 1)
+mma_kernel(int n, int issuers, int count, int wait_every, unsigned long long* cycles, int* err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5;
+  const uint32_t done = base + 64, ready = base + 72, a_s = base + 1024, b_s = base + 1024 + 16384;
+  for (int i = threadIdx.x; i < (16384 + 32768) / 16; i += 128) st_shared_v4(a_s + i * 16, 0u, 0u, 0u, 0u);
+  if (threadIdx.x == 0) {
+    mbar_init(done, 1);
+    mbar_init(done + 16, 1);
+    mbar_init(ready, 1);
+    fence_mbar_init();
+    mbar_arrive(ready);                  // phase 0 of `ready` is complete from the start
+  }
+  fence_proxy_async_cta();
+  if (warp == 0) {
+    tmem_alloc(base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + (base - smem_u32(smem_raw)));
+  // issuer w (lane 0 of warp w < issuers) accumulates into TMEM columns [w n, (w + 1) n), takes
+  // A from TMEM columns 256 + 128 w on (or from the shared A tile, which both only read), and
+  // issues count / issuers MMAs
+  const int lane = threadIdx.x & 31;
+  if (lane == 0 && warp < issuers) {
+    const uint32_t idesc = ((1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+                            ((uint32_t)(128 >> 4) << 24));
+    const uint32_t d = tmem + (uint32_t)(warp * n), a_t = tmem + 256 + warp * 128;
+    // descriptors formed before the clock starts; 4 MMAs (one 64-column K chunk) per loop
+    // trip, and the wait cadence kept by a countdown rather than a division
+    uint64_t ad[4], bd[4];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      ad[kk] = smem_desc_sw128(a_s + kk * 32, 16, 1024);
+      bd[kk] = smem_desc_sw128(b_s + kk * 32, 16, 1024);
+    }
+    const int mine = count / issuers;
+    const uint32_t bar = done + 16u * warp;
+    int left = wait_every;
+    const long long t0 = clock64();
+    for (int i = 0; i < mine; i += 4) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
+        if (A_TMEM) mma_bf16_ts(d, a_t + kk * 8, bd[kk], idesc, acc);
+        else mma_bf16_ss(d, ad[kk], bd[kk], idesc, acc);
+      }
+      if (wait_every > 0 && (left -= 4) <= 0) {
+        (void)mbar_try_wait(ready, 0);
+        left = wait_every;
+      }
+    }
+    tc_commit(bar);
+    bool ok = poll(bar, 0, false);
+    const long long t1 = clock64();
+    if (!ok) {                           // MMAs always finish: wait again (bounded) before freeing TMEM
+      atomicOr(err, 1);
+      poll(bar, 0, false);
+    }
+    atomicMax(cycles + blockIdx.x, (unsigned long long)(t1 - t0));
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static std::once_flag once;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -292,4 +376,24 @@ extern "C" int kd_probe_store(void* buf, int ctas, int mode, int reps, unsigned 
     return st;
   store_kernel<<<ctas, 256, smem, stream>>>(tm, static_cast<float*>(buf), mode, reps, cycles);
   return kd::launch_status("store probe");
+}
+
+// n in {64, 128, 256}; a_tmem 0 / 1; issuers 1, or 2 with n <= 128 (each its own accumulator);
+// count in [4 issuers, 2^22] and wait_every >= 0, multiples of 4 (count of 4 issuers).  cycles:
+// device uint64 [148], zeroed by the caller (the slower issuer's time per CTA); err: device
+// int32 (ORed; set if a final wait gave up once).  Grid: 148 CTAs.
+extern "C" int kd_probe_mma(int n, int a_tmem, int issuers, int count, int wait_every, unsigned long long* cycles,
+                            int* err, cudaStream_t stream) {
+  using namespace kd::probe;
+  if (!cycles || !err || (n != 64 && n != 128 && n != 256) || (a_tmem != 0 && a_tmem != 1) ||
+      (issuers != 1 && issuers != 2) || (issuers == 2 && n > 128) || count < 4 * issuers || count > (1 << 22) ||
+      count % (4 * issuers) || wait_every < 0 || (wait_every & 3))
+    return KD_EINVAL;
+  int st;
+  auto kern = a_tmem ? mma_kernel<true> : mma_kernel<false>;
+  if ((st = kd::cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MMA_SMEM),
+                            "cudaFuncSetAttribute(mma probe)")))
+    return st;
+  kern<<<148, 128, MMA_SMEM, stream>>>(n, issuers, count, wait_every, cycles, err);
+  return kd::launch_status("mma probe");
 }
