@@ -27,12 +27,16 @@
 //       the row max on raw scores, keep an online max with a lazy rescale
 //       threshold, and emit P as two 128-key halves: each half is written into a
 //       local staging slot in the K-major swizzled layout the MMA reads and moved
-//       to rank 1 by a single bulk copy that completes on rank 1's barrier.
+//       to rank 1 by a single bulk copy that completes on rank 1's barrier.  A tile
+//       whose second half lies past the request's last key is computed by N=128
+//       MMAs and sends only its first half.
 //   rank 1 ("PV" CTA): O (128 x 512 fp32) in TMEM; V as 64-key x 256-column
 //       groups (four 64-column MN-major boxes) in a 4-deep ring; O += P V as
 //       M=128, N=256, K=16 MMAs; V groups wholly past the request's last key are
 //       neither loaded nor multiplied.  Two 4-warp groups apply the rare O rescale
-//       and write the normalised output straight from registers to global memory.
+//       and write the normalised output (or a split's fp32 partial) as TMA box
+//       stores staged through shared memory; a cluster's last unit stages through
+//       the then idle P slots and V ring, many boxes in flight.
 //
 // The kernel is persistent: one cluster per SM pair.  Units are handed out
 // dynamically from a global counter in longest-request-first order; each cluster's
