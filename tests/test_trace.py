@@ -80,13 +80,16 @@ def test_mma_probe_runs(kd, traced):
     trace, lib, product, dims = traced
     cycles = torch.zeros(148, dtype=torch.int64, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for n, a_tmem, issuers, wait_every in [(64, 0, 1, 0), (256, 1, 1, 0), (128, 1, 2, 0), (128, 1, 1, 4)]:
+    for m, n, a_tmem, issuers, wait_every in [(128, 64, 0, 1, 0), (128, 256, 1, 1, 0), (128, 128, 1, 2, 0),
+                                              (128, 128, 1, 1, 4), (64, 256, 0, 1, 0)]:
         cycles.zero_()
-        rc = lib.kd_probe_mma(n, a_tmem, issuers, 64, wait_every, cycles.data_ptr(), err.data_ptr(),
+        rc = lib.kd_probe_mma(m, n, a_tmem, issuers, 64, wait_every, cycles.data_ptr(), err.data_ptr(),
                               torch.cuda.current_stream().cuda_stream)
         assert rc == 0
         torch.cuda.synchronize()
         assert int(err.item()) == 0
         assert (cycles.cpu().numpy() > 0).all()
-    assert lib.kd_probe_mma(96, 0, 1, 64, 0, cycles.data_ptr(), err.data_ptr(), None) != 0
-    assert lib.kd_probe_mma(256, 1, 2, 64, 0, cycles.data_ptr(), err.data_ptr(), None) != 0
+    assert lib.kd_probe_mma(128, 96, 0, 1, 64, 0, cycles.data_ptr(), err.data_ptr(), None) != 0
+    assert lib.kd_probe_mma(128, 256, 1, 2, 64, 0, cycles.data_ptr(), err.data_ptr(), None) != 0
+    assert lib.kd_probe_mma(32, 128, 0, 1, 64, 0, cycles.data_ptr(), err.data_ptr(), None) != 0
+    assert lib.kd_probe_mma(64, 128, 1, 1, 64, 0, cycles.data_ptr(), err.data_ptr(), None) != 0

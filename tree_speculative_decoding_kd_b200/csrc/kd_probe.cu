@@ -22,7 +22,7 @@
 //     contiguous bytes of a row.
 //
 // kd_probe_mma measures the tensor pipe as its issuing threads see it: each CTA (one per SM)
-// issues `count` tcgen05.mma (kind::f16, bf16, M = 128, K = 16, N = 64 / 128 / 256) back to back
+// issues `count` tcgen05.mma (kind::f16, bf16, M = 64 or 128, K = 16, N = 64 / 128 / 256) back to back
 // from one thread (or from two threads in two warps, each into its own accumulator) into TMEM,
 // A from shared memory or from TMEM, B from shared memory, and with
 // `wait_every` > 0 it polls an already-completed mbarrier after every `wait_every` MMAs (a
@@ -225,7 +225,7 @@ store_kernel(const __grid_constant__ CUtensorMap tm, float* buf, int mode, int r
 constexpr int MMA_SMEM = 120 * 1024;
 template <bool A_TMEM>
 __global__ void __launch_bounds__(128, 1)
-mma_kernel(int n, int issuers, int count, int wait_every, unsigned long long* cycles, int* err) {
+mma_kernel(int m, int n, int issuers, int count, int wait_every, unsigned long long* cycles, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5;
@@ -253,7 +253,7 @@ mma_kernel(int n, int issuers, int count, int wait_every, unsigned long long* cy
   const int lane = threadIdx.x & 31;
   if (lane == 0 && warp < issuers) {
     const uint32_t idesc = ((1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
-                            ((uint32_t)(128 >> 4) << 24));
+                            ((uint32_t)(m >> 4) << 24));
     const uint32_t d = tmem + (uint32_t)(warp * n), a_t = tmem + 256 + warp * 128;
     // descriptors formed before the clock starts; 4 MMAs (one 64-column K chunk) per loop
     // trip, and the wait cadence kept by a countdown rather than a division
@@ -378,14 +378,16 @@ extern "C" int kd_probe_store(void* buf, int ctas, int mode, int reps, unsigned 
   return kd::launch_status("store probe");
 }
 
-// n in {64, 128, 256}; a_tmem 0 / 1; issuers 1, or 2 with n <= 128 (each its own accumulator);
+// m in {64, 128} (64 with A from shared memory only); n in {64, 128, 256}; a_tmem 0 / 1; issuers 1,
+// or 2 with n <= 128 (each its own accumulator);
 // count in [4 issuers, 2^22] and wait_every >= 0, multiples of 4 (count of 4 issuers).  cycles:
 // device uint64 [148], zeroed by the caller (the slower issuer's time per CTA); err: device
 // int32 (ORed; set if a final wait gave up once).  Grid: 148 CTAs.
-extern "C" int kd_probe_mma(int n, int a_tmem, int issuers, int count, int wait_every, unsigned long long* cycles,
-                            int* err, cudaStream_t stream) {
+extern "C" int kd_probe_mma(int m, int n, int a_tmem, int issuers, int count, int wait_every,
+                            unsigned long long* cycles, int* err, cudaStream_t stream) {
   using namespace kd::probe;
-  if (!cycles || !err || (n != 64 && n != 128 && n != 256) || (a_tmem != 0 && a_tmem != 1) ||
+  if (!cycles || !err || (m != 64 && m != 128) || (n != 64 && n != 128 && n != 256) || (a_tmem != 0 && a_tmem != 1) ||
+      (m == 64 && a_tmem) ||
       (issuers != 1 && issuers != 2) || (issuers == 2 && n > 128) || count < 4 * issuers || count > (1 << 22) ||
       count % (4 * issuers) || wait_every < 0 || (wait_every & 3))
     return KD_EINVAL;
@@ -394,6 +396,6 @@ extern "C" int kd_probe_mma(int n, int a_tmem, int issuers, int count, int wait_
   if ((st = kd::cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MMA_SMEM),
                             "cudaFuncSetAttribute(mma probe)")))
     return st;
-  kern<<<148, 128, MMA_SMEM, stream>>>(n, issuers, count, wait_every, cycles, err);
+  kern<<<148, 128, MMA_SMEM, stream>>>(m, n, issuers, count, wait_every, cycles, err);
   return kd::launch_status("mma probe");
 }

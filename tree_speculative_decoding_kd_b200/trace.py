@@ -80,7 +80,7 @@ def _load():
                                       ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
     lib.kd_probe_store.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                    ctypes.c_void_p]
-    lib.kd_probe_mma.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+    lib.kd_probe_mma.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
     c, s = ctypes.c_int(), ctypes.c_int()
     lib.kd_trace_dims(ctypes.byref(c), ctypes.byref(s))
@@ -235,16 +235,17 @@ def probes(lib, iters=3000):
 
 
 def mma_probes(lib, count=4096):
-    """Dense FLOP per SM cycle of M=128 K=16 bf16 MMAs from one or two issuing threads per SM."""
+    """Dense FLOP per SM cycle of M=128 (or 64) K=16 bf16 MMAs from one or two issuing threads per SM."""
     cycles = torch.zeros(148, dtype=torch.int64, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    cases = [(n, a, 1, 0) for n in (64, 128, 256) for a in (0, 1)] + \
-            [(n, 1, 2, 0) for n in (64, 128)] + [(n, 1, 1, w) for n in (128, 256) for w in (4, 36)]
+    cases = [(128, n, a, 1, 0) for n in (64, 128, 256) for a in (0, 1)] + \
+            [(128, n, 1, 2, 0) for n in (64, 128)] + [(128, n, 1, 1, w) for n in (128, 256) for w in (4, 36)] + \
+            [(64, n, 0, 1, 0) for n in (128, 256)]
     out = []
-    for n, a_tmem, issuers, wait_every in cases:
+    for m, n, a_tmem, issuers, wait_every in cases:
         for _ in range(2):
             cycles.zero_()
-            rc = lib.kd_probe_mma(n, a_tmem, issuers, count, wait_every, cycles.data_ptr(), err.data_ptr(),
+            rc = lib.kd_probe_mma(m, n, a_tmem, issuers, count, wait_every, cycles.data_ptr(), err.data_ptr(),
                                   torch.cuda.current_stream().cuda_stream)
             if rc != 0:
                 raise RuntimeError(f"mma probe rc {rc}")
@@ -252,10 +253,10 @@ def mma_probes(lib, count=4096):
         if int(err.item()) != 0:
             raise RuntimeError("an mma probe wait gave up")
         cyc = float(np.median(cycles.cpu().numpy().astype(np.float64)))
-        out.append({"probe": "mma", "N": n, "A": "tmem" if a_tmem else "smem", "issuers": issuers,
+        out.append({"probe": "mma", "M": m, "N": n, "A": "tmem" if a_tmem else "smem", "issuers": issuers,
                     "wait_every": wait_every or None,
                     "cycles_per_mma_per_issuer": round(cyc / (count // issuers), 1),
-                    "FLOP_per_SM_cycle_median": round(count * 2.0 * 128 * n * 16 / cyc, 0)})
+                    "FLOP_per_SM_cycle_median": round(count * 2.0 * m * n * 16 / cyc, 0)})
     return out
 
 
