@@ -276,6 +276,20 @@ def test_attn_ragged_and_edge_shapes(kd, L_lo, L_hi, n, H):
     assert_attn(out, lse, ro, rl, f"edge {L_lo}-{L_hi} n{n} H{H}")
 
 
+@pytest.mark.parametrize("kv_splits", [0, 2])
+def test_attn_more_requests_than_the_longest_first_table(kd, kv_splits):
+    """300 requests (more than the kernel's 256-entry longest-first table, so units go in
+    request order), each with its own length, some with no committed keys; automatic and
+    forced key partitions."""
+    cfg = W.Config("many", 300, 2, 2, 0, 300, "uniform", 0, 91)
+    wl = W.make_workload(cfg)
+    wl.cache_lens[::37] = 0                     # tree-only requests among them
+    out, lse, bits = run_attn(kd, wl, kv_splits=kv_splits)
+    ro, rl = oracle_attn(wl)
+    assert bits == 0
+    assert_attn(out, lse, ro, rl, f"B=300 splits={kv_splits}")
+
+
 @pytest.mark.parametrize("mul", [16.0, 64.0])
 def test_attn_peaked_softmax_with_rescales(kd, mul):
     """Large scale makes the softmax peaked and forces running-max rescales."""
