@@ -208,11 +208,9 @@ class Verifier:
         self.path = torch.empty(B, n, dtype=torch.int32, device=dev)
         self.len = torch.empty(B, dtype=torch.int32, device=dev)
         self.bonus = torch.empty(B, dtype=torch.int32, device=dev)
-        self.launches_per_step = 5 + (1 if self._splits() > 1 else 0)
-
-    def _splits(self):
-        return 1 if self.kd.kd_verify_workspace_bytes(self.cfg.B, self.cfg.n, self.cfg.H,
-                                                      self.cfg.cap, 0) <= 256 else 2
+        # node write, mask, attention (its split-KV merge runs inside the same launch),
+        # accept, compaction
+        self.launches_per_step = 5
 
     def step(self, s: DeviceStep, ev=None):
         kd = self.kd
@@ -442,11 +440,13 @@ def run_kd(args):
     # cache lengths each timed step starts from: the generator knows every
     # step's accepted length (its planted path), so no device copy is timed
     lens_np = wl.cache_lens.astype(np.int64).copy()
-    step_lens = []
+    step_lens, drafts = [], []
     for s in range(args.warmup + args.steps):
+        planted = [len(p) for p in host_steps[s % N_DISTINCT].planted]
         if s >= args.warmup:
             step_lens.append(lens_np.copy())
-        lens_np += np.array([len(p) for p in host_steps[s % N_DISTINCT].planted])
+            drafts += [k - 1 for k in planted]             # accepted drafts (the root excluded)
+        lens_np += np.array(planted)
     attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
     HN.barrier(local)
@@ -572,7 +572,12 @@ def run_kd(args):
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": V.launches_per_step * args.steps,
                 "clocks": clk.summary(),
-                "device_errors": err_bits}
+                "device_errors": err_bits,
+                "accepted_drafts": {"mean": round(float(np.mean(drafts)), 3),
+                                    "histogram": {str(k): int(v) for k, v in
+                                                  zip(*np.unique(drafts, return_counts=True))},
+                                    "source": "the timed steps' planted paths (per request and step); "
+                                              "the device's cache lengths after the run equal their sums"}}
         if cpu is not None:
             line["cpu_baseline"] = cpu
         if extras is not None:
