@@ -61,7 +61,7 @@ argmax_accept_kernel(const float* __restrict__ logits, int64_t V, int chunks, in
   const float4* src = reinterpret_cast<const float4*>(logits + row * V);
   const int64_t e0 = (int64_t)chunk * AM_CHUNK + (int64_t)threadIdx.x * 4;
 
-  // all eight loads first (V is a multiple of 4, so a vector is either wholly inside
+  // all sixteen loads first (V is a multiple of 4, so a vector is either wholly inside
   // the row or wholly past its end; past the end reads as -inf and is never chosen)
   const float NEG = -INFINITY;
   float4 x[AM_VEC];
