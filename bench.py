@@ -316,12 +316,30 @@ def accept_logits_case(kd, torch, peaks, name="loop", reps=10, warm=3, requests=
     ok = bool((am.cpu().numpy() == st.argmax[:R]).all())
     t = float(np.median(times))
     nbytes = B * n * V * 4
-    del logits
+    # for scale: PyTorch's own row reductions over the same tensor, timed the same way
+    # (library kernels, outside every other timed region)
+    flat = logits.view(B * n, V)
+    ref = {}
+    for rname, fn in (("torch_amax", lambda: torch.amax(flat, dim=-1)),
+                      ("torch_argmax", lambda: torch.argmax(flat, dim=-1))):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        rt = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            rt.append(e0.elapsed_time(e1) * 1e-3)
+        ref[rname + "_us"] = round(float(np.median(rt)) * 1e6, 2)
+    del logits, flat
     torch.cuda.empty_cache()
     return {"workload": f"{name}: {B} requests x {n} nodes x {V} fp32 logits", "us": round(t * 1e6, 2),
             "us_min": round(min(times) * 1e6, 2), "hbm_gbs": round(nbytes / t / 1e9, 1),
             "roofline_frac": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 3), "bound": "hbm",
-            "bytes": nbytes, "planted_tokens_recovered": ok,
+            "bytes": nbytes, "planted_tokens_recovered": ok, "library_reference": ref,
             "timing": "CUDA events around each call; logits larger than L2, so no flush"}
 
 
