@@ -71,6 +71,8 @@ def parse():
     ap.add_argument("--attn-only", default=None, choices=["tiny", "kimi_single", "batched", "long", "extend"],
                     help="time only the attention of one single-step configuration")
     ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--gemm-reference", action="store_true",
+                    help="with --attn-only batched/long: also time the two plain GEMMs by torch.matmul")
     ap.add_argument("--accept-logits-only", action="store_true",
                     help="time only the fused target argmax + accept on the loop workload's trees")
     ap.add_argument("--requests", type=int, default=0,
@@ -276,10 +278,61 @@ def attn_case(kd, torch, peaks, flush, name, reps=20, warm=3):
     return res
 
 
+def gemm_reference(kd, torch, flush, name, reps=10, warm=2):
+    """For scale: the two plain contractions of the attention, S = Q K^T (bf16 out) and
+    O = S V per request, by torch.matmul (cuBLAS) on the same inputs: no mask, no softmax,
+    S through memory.  Timed like attn_case (CUDA-graph replay after an L2 flush)."""
+    wl = W.make_workload(name)
+    cfg, st = wl.cfg, wl.step
+    B, n, H = cfg.B, cfg.n, cfg.H
+    bf = torch.bfloat16
+    q = torch.cat([kd.bf16_from_bits(st.q_abs), kd.bf16_from_bits(st.q_rope)], dim=-1).reshape(B, n * H, 576)
+    # key counts rounded up to 64 (zero rows past the cache), so that every operand row
+    # is 16-byte aligned, as cuBLAS's tensor-core kernels want
+    cap_pad = (cfg.cap + 63) // 64 * 64
+    kv = torch.zeros(B, cap_pad, 576, dtype=bf, device="cuda")
+    kv[:, :cfg.cap] = torch.cat([kd.bf16_from_bits(wl.c_kv), kd.bf16_from_bits(wl.k_rope)], dim=-1)
+    keys = [(int(wl.cache_lens[b]) + n + 63) // 64 * 64 for b in range(B)]
+    S = [torch.empty(n * H, keys[b], dtype=bf, device="cuda") for b in range(B)]
+    O = [torch.empty(n * H, 512, dtype=bf, device="cuda") for b in range(B)]
+
+    def call():
+        for b in range(B):
+            torch.matmul(q[b], kv[b, :keys[b]].t(), out=S[b])
+            torch.matmul(S[b], kv[b, :keys[b], :512], out=O[b])
+
+    for _ in range(warm):
+        call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    times = []
+    for _ in range(reps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3)
+    del graph, q, kv, S, O
+    torch.cuda.empty_cache()
+    t = float(np.median(times))
+    flops = sum(2.0 * n * H * k * (576 + 512) for k in keys)
+    return {"torch_matmul_qk_then_sv_us": round(t * 1e6, 2), "tflops": round(flops / t / 1e12, 1),
+            "what": "S = Q K^T (bf16) then O = S V per request, torch.matmul (cuBLAS), no mask or "
+                    "softmax, every key pair computed (keys rounded up to 64)"}
+
+
 def attn_extras(kd, torch, peaks, flush):
-    """Attention-only timings of the single-step configurations (parity cases)."""
-    return {name: attn_case(kd, torch, peaks, flush, name) for name in
-            ["tiny", "kimi_single", "batched", "long"]}
+    """Attention-only timings of the single-step configurations (parity cases), with the
+    plain two-GEMM time of the large ones for scale."""
+    res = {name: attn_case(kd, torch, peaks, flush, name) for name in
+           ["tiny", "kimi_single", "batched", "long"]}
+    for name in ("batched", "long"):
+        res[name]["library_reference"] = gemm_reference(kd, torch, flush, name)
+    return res
 
 
 def accept_logits_case(kd, torch, peaks, name="loop", reps=10, warm=3, requests=0):
@@ -428,7 +481,10 @@ def run_attn_only(args):
     torch.cuda.set_device(0)
     from tree_speculative_decoding_kd_b200 import kd
     peaks = HN.load_peaks(ROOT)
-    res = attn_case(kd, torch, peaks, HN.L2Flush("cuda"), args.attn_only, reps=args.reps, warm=1)
+    flush = HN.L2Flush("cuda")
+    res = attn_case(kd, torch, peaks, flush, args.attn_only, reps=args.reps, warm=1)
+    if args.attn_only in ("batched", "long") and args.gemm_reference:
+        res["library_reference"] = gemm_reference(kd, torch, flush, args.attn_only)
     print(json.dumps({"attn_only": args.attn_only, **res}), flush=True)
 
 
