@@ -276,6 +276,35 @@ def test_attn_ragged_and_edge_shapes(kd, L_lo, L_hi, n, H):
     assert_attn(out, lse, ro, rl, f"edge {L_lo}-{L_hi} n{n} H{H}")
 
 
+def test_a_wait_that_runs_out_reports_and_leaves_the_context_usable(kd):
+    """Failure detection without a fault: the first M tile's merge ticket is planted far
+    below its partition count, so the CTAs merging that tile wait for partials that never
+    complete it.  Their bounded wait gives up after the kernel's 2-second limit, raises
+    KD_DEV_TIMEOUT, records where in the control block, and every role leaves; once the
+    workspace is cleared, the next call on the same context is correct."""
+    cfg = W.Config("timeout", 1, 16, 8, 300, 300, "uniform", 0, 93)   # 308 keys: 2 partitions
+    wl = W.make_workload(cfg)
+    st = wl.step
+    args = (dev_bf16(kd, st.q_abs), dev_bf16(kd, st.q_rope), dev_bf16(kd, wl.c_kv),
+            dev_bf16(kd, wl.k_rope), dev_i32(wl.cache_lens))
+    vis = torch.from_numpy(vis_for(st.parents).view(np.int32)).cuda()
+    ws = kd.new_workspace(1, cfg.n, cfg.H, cfg.cap, 2)
+    words = ws.view(torch.int32)
+    words[256 // 4] = -1000                     # the first M tile's ticket (after the control block)
+    kd.kd_tree_verify_attn(*args, vis, None, cfg.scale, workspace=ws, kv_splits=2)
+    torch.cuda.synchronize()
+    site = int(words[1].item())
+    assert kd.kd_read_device_error(ws) & 0x10, "KD_DEV_TIMEOUT expected"
+    assert site & (1 << 31), "the wait that gave up is recorded at byte 4"
+    ws.zero_()
+    out, lse = kd.kd_tree_verify_attn(*args, vis, None, cfg.scale, workspace=ws, kv_splits=2)
+    torch.cuda.synchronize()
+    assert kd.kd_read_device_error(ws) == 0
+    o = kd.bits_from_bf16(out)
+    ro, rl = oracle_attn(wl)
+    assert_attn((o.astype(np.uint32) << 16).view(np.float32), lse.cpu().numpy(), ro, rl, "after a timeout")
+
+
 @pytest.mark.parametrize("kv_splits", [0, 2])
 def test_attn_more_requests_than_the_longest_first_table(kd, kv_splits):
     """300 requests (more than the kernel's 256-entry longest-first table, so units go in
