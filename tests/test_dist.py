@@ -58,6 +58,49 @@ def test_two_ranks_weak_scaling_and_max_timing():
     assert env0 == (0, 2, 0) and env1 == (1, 2, 1)
 
 
+def _dying_worker(rank, world, port, q):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import time
+    import torch.distributed as dist
+    HN.init_dist("gloo", timeout_s=5)
+    HN.barrier()                                        # both ranks start the run together
+    if rank == 1:
+        q.put((1, "left"))                              # rank 1 dies between steps
+        q.close()
+        q.join_thread()                                 # (the message is sent before the exit)
+        os._exit(0)
+    t0 = time.monotonic()
+    try:
+        HN.barrier()                                    # the next step's barrier never completes
+        q.put((0, "passed"))
+    except Exception as e:                              # the short process-group timeout ends it
+        q.put((0, f"error after {time.monotonic() - t0:.1f} s: {type(e).__name__}"))
+    finally:
+        try:
+            dist.destroy_process_group()
+        except Exception:
+            pass
+
+
+def test_a_rank_that_dies_between_steps_ends_the_others_with_an_error():
+    """A rank that leaves between steps (no kernel or collective of it in flight): the
+    surviving rank's next barrier ends with an error at the process group's short
+    timeout instead of waiting for good."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+    assert res[1] == "left"
+    assert res[0].startswith("error after"), res[0]
+    assert float(res[0].split()[2]) < 60.0
+
+
 def test_single_process_defaults():
     for k in ["RANK", "WORLD_SIZE", "LOCAL_RANK"]:
         os.environ.pop(k, None)
