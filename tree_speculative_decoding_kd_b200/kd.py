@@ -197,9 +197,11 @@ def kd_tree_verify_attn_simt(q_abs, q_rope, c_kv, k_rope, cache_lens, vis, posit
     return out, lse
 
 
-def kd_tree_build(logp, cand_tokens, root_tokens, n, stream=None):
+def kd_tree_build(logp, cand_tokens, root_tokens, n, parents=None, tokens=None, depth=None, score=None,
+                  stream=None):
     """Best-first draft trees: logp fp32 [B][D][K] (sorted per depth), cand_tokens int32
-    [B][D][K], root_tokens int32 [B] -> (parents, tokens, depth, score), each [B][n]."""
+    [B][D][K], root_tokens int32 [B] -> (parents, tokens, depth, score), each [B][n]
+    (allocated here unless given)."""
     _need(logp, torch.float32, "logp")
     _need(cand_tokens, torch.int32, "cand_tokens")
     _need(root_tokens, torch.int32, "root_tokens")
@@ -207,10 +209,19 @@ def kd_tree_build(logp, cand_tokens, root_tokens, n, stream=None):
     if tuple(cand_tokens.shape) != (B, D, K) or tuple(root_tokens.shape) != (B,):
         raise ValueError("cand_tokens must be [B][D][K] and root_tokens [B]")
     dev = logp.device
-    parents = torch.empty(B, n, dtype=torch.int32, device=dev)
-    tokens = torch.empty(B, n, dtype=torch.int32, device=dev)
-    depth = torch.empty(B, n, dtype=torch.int32, device=dev)
-    score = torch.empty(B, n, dtype=torch.float32, device=dev)
+    if parents is None:
+        parents = torch.empty(B, n, dtype=torch.int32, device=dev)
+    if tokens is None:
+        tokens = torch.empty(B, n, dtype=torch.int32, device=dev)
+    if depth is None:
+        depth = torch.empty(B, n, dtype=torch.int32, device=dev)
+    if score is None:
+        score = torch.empty(B, n, dtype=torch.float32, device=dev)
+    for t, dt, name in ((parents, torch.int32, "parents"), (tokens, torch.int32, "tokens"),
+                        (depth, torch.int32, "depth"), (score, torch.float32, "score")):
+        _need(t, dt, name)
+        if tuple(t.shape) != (B, n):
+            raise ValueError(f"{name} must be [B][n]")
     _check(lib.kd_tree_build(_ptr(logp), _ptr(cand_tokens), _ptr(root_tokens), B, D, K, n,
                              _ptr(parents), _ptr(tokens), _ptr(depth), _ptr(score), _stream(stream)),
            "kd_tree_build")
