@@ -30,7 +30,7 @@ def check(kd, logp, toks, root, n):
 
 @pytest.mark.parametrize("B,D,K,n", [(3, 4, 3, 30), (5, 16, 8, 17), (4, 1, 8, 9), (2, 6, 1, 7),
                                      (2, 127, 2, 128), (2, 2, 255, 128), (33, 8, 4, 64),
-                                     (2, 64, 32, 128)])     # the last: too large to stage, read in place
+                                     (2, 64, 32, 128)])     # the last: a large candidate table
 def test_tree_build_random(kd, B, D, K, n):
     rng = np.random.default_rng(D * 1000 + K * 10 + n)
     check(kd, *cands(rng, B, D, K), n)
